@@ -1,0 +1,473 @@
+#!/usr/bin/env python3
+"""Benchmark of the paged-attention hot path on B200.
+
+One step = the whole path over one batch: write the step's new K/V rows into
+the paged pool (pa_reshape_and_cache), then paged attention over every
+sequence's cached context (pa_decode; pa_varlen for the mixed step).  The
+default workload is the LLaMA-13B-shaped MHA decode: 64 sequences, context
+lengths uniform in [128, 2048], 40 heads of dimension 128, bf16, 16-token
+blocks in a 12000-block pool.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 2..5] [--impl reference]
+
+Rank 0 prints one JSON line.  Under torchrun every rank runs an independent
+replica of the workload (the path has no exchange step), timed on the device
+and reduced as the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paged_kv_cache_lens_b200 import workloads as wl  # noqa: E402
+
+METRIC = "paged decode attention: achieved HBM GB/s (% of peak), sequence-steps/s/layer"
+FALLBACK_HBM_GBS = 6650.0
+CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", type=int, default=2, choices=[2, 3, 4, 5])
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def algorithmic_bytes(W) -> dict:
+    """Bytes the step must move at least once: every visible key and value of
+    every (request, KV head), the queries, the outputs, the block-table
+    entries read, and the new rows written (read + write)."""
+    kv = W.kv_bytes_read()
+    q = W.total_q * W.num_q_heads * W.head_dim * 2
+    out = W.total_q * W.num_q_heads * W.head_dim * (4 if W.out_dtype == wl.F32 else 2)
+    tbl = int((-(-W.seqlens_k.astype(np.int64) // W.block_size)).sum()) * 4 + W.num_seqs * 4
+    new = int((W.new_slots >= 0).sum()) * W.num_kv_heads * W.head_dim * 2 * (
+        2 + W.kv_elem_bytes()) + W.total_q * 8
+    return {"kv": kv, "attention": kv + q + out + tbl, "step": kv + q + out + tbl + new}
+
+
+def workload_name(W) -> str:
+    return wl.CONFIG_NAMES[int(W.name[6])] if W.name.startswith("config") else W.name
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={CLOCK_QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                    rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows]
+        mx = [float(r[2]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": reasons,
+                "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------
+# distributed plumbing (replicas only)
+# --------------------------------------------------------------------------
+
+def dist_setup(n_gpus):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------
+# the native arm
+# --------------------------------------------------------------------------
+
+def run_native(args):
+    import torch
+    from paged_kv_cache_lens_b200 import pa
+
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local if world > 1 else 0)
+    W = wl.config(args.workload)
+    TD = {wl.F16: torch.float16, wl.BF16: torch.bfloat16, wl.F32: torch.float32}
+
+    def to_dev(a, dt):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(TD[dt])
+
+    shape = (W.num_blocks, W.num_kv_heads, W.block_size, W.head_dim)
+    if W.kv_dtype == wl.FP8_E4M3:
+        kc = torch.zeros(shape, dtype=torch.uint8, device=dev)
+        vc = torch.zeros(shape, dtype=torch.uint8, device=dev)
+        ks = torch.from_numpy(W.k_scale).to(dev)
+        vs = torch.from_numpy(W.v_scale).to(dev)
+    else:
+        kc = torch.zeros(shape, dtype=TD[W.kv_dtype], device=dev)
+        vc = torch.zeros(shape, dtype=TD[W.kv_dtype], device=dev)
+        ks = vs = None
+    stream = torch.cuda.current_stream(dev)
+    # cached context (setup, untimed)
+    chunk = 1 << 18
+    for s in range(0, len(W.prefill_slots), chunk):
+        e = min(len(W.prefill_slots), s + chunk)
+        pa.pa_reshape_and_cache(to_dev(W.prefill_k[s:e], W.src_dtype),
+                                to_dev(W.prefill_v[s:e], W.src_dtype),
+                                torch.from_numpy(W.prefill_slots[s:e]).to(dev), kc, vc, ks, vs)
+    torch.cuda.synchronize(dev)
+
+    # step inputs resident in HBM
+    q = to_dev(W.q, W.q_dtype)
+    nk, nv = to_dev(W.new_k, W.src_dtype), to_dev(W.new_v, W.src_dtype)
+    slots = torch.from_numpy(W.new_slots).to(dev)
+    bt = torch.from_numpy(W.block_tables).to(dev)
+    sk = torch.from_numpy(W.seqlens_k).to(dev)
+    cu = torch.from_numpy(W.cu_seqlens_q).to(dev)
+    out = torch.empty((W.total_q, W.num_q_heads, W.head_dim), dtype=TD[W.out_dtype], device=dev)
+    if W.decode:
+        nws = pa.pa_decode_workspace_size(W.num_seqs, W.num_q_heads, W.head_dim,
+                                          W.max_context_len, W.partition_size)
+    else:
+        nws = pa.pa_varlen_workspace_size(W.num_seqs, W.total_q, W.num_q_heads, W.head_dim,
+                                          W.max_context_len)
+    ws = torch.empty(max(nws, 256), dtype=torch.uint8, device=dev)
+
+    def attend(q_, bt_, sk_, cu_, out_):
+        if W.decode:
+            pa.pa_decode(out_, q_, kc, vc, bt_, sk_, W.max_context_len, W.scale, ks, vs,
+                         W.partition_size, ws, stream)
+        else:
+            pa.pa_varlen(out_, q_, cu_, sk_, W.max_q_len, W.max_context_len, kc, vc, bt_,
+                         W.scale, ks, vs, ws, stream)
+
+    def step():
+        pa.pa_reshape_and_cache(nk, nv, slots, kc, vc, ks, vs, stream)
+        attend(q, bt, sk, cu, out)
+
+    max_parts = -(-W.max_context_len // (W.partition_size or 512))
+    launches_per_step = 1 + 1 + (1 if max_parts > 1 else 0) + (0 if W.decode else 1)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+
+    # ---- device-timed region: K whole steps, attention launches timed too
+    ev_a = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        t0.record(stream)
+        for i in range(args.steps):
+            pa.pa_reshape_and_cache(nk, nv, slots, kc, vc, ks, vs, stream)
+            ev_a[i][0].record(stream)
+            attend(q, bt, sk, cu, out)
+            ev_a[i][1].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+    ms_local = t0.elapsed_time(t1) / args.steps
+    attn_ms = float(np.mean([a.elapsed_time(b) for a, b in ev_a]))
+    ms = max_over_ranks(ms_local, world)
+    attn_ms = max_over_ranks(attn_ms, world)
+    assert pa.pa_device_error(stream) == 0
+
+    # ---- end to end through the public API from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()  # noqa: E731
+        h_q = pin(W.q.view(np.int16))
+        h_k, h_v = pin(W.new_k.view(np.int16)), pin(W.new_v.view(np.int16))
+        h_slots, h_bt = pin(W.new_slots), pin(W.block_tables)
+        h_sk, h_cu = pin(W.seqlens_k), pin(W.cu_seqlens_q)
+        h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        d_q, d_k, d_v = torch.empty_like(q), torch.empty_like(nk), torch.empty_like(nv)
+        d_slots, d_bt, d_sk, d_cu = (torch.empty_like(slots), torch.empty_like(bt),
+                                     torch.empty_like(sk), torch.empty_like(cu))
+        h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_slots, h_bt, h_sk, h_cu))
+        d2h = h_out.numel() * h_out.element_size()
+
+        def e2e_step():
+            d_q.view(torch.int16).copy_(h_q, non_blocking=True)
+            d_k.view(torch.int16).copy_(h_k, non_blocking=True)
+            d_v.view(torch.int16).copy_(h_v, non_blocking=True)
+            d_slots.copy_(h_slots, non_blocking=True)
+            d_bt.copy_(h_bt, non_blocking=True)
+            d_sk.copy_(h_sk, non_blocking=True)
+            d_cu.copy_(h_cu, non_blocking=True)
+            pa.pa_reshape_and_cache(d_k, d_v, d_slots, kc, vc, ks, vs, stream)
+            attend(d_q, d_bt, d_sk, d_cu, out)
+            h_out.copy_(out, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
+        e2e = (e2e_ms, h2d, d2h)
+
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    by = algorithmic_bytes(W)
+    peak, peak_kind = peaks()
+    gbs = by["kv"] * world / (ms * 1e-3) / 1e9
+    attn_gbs = by["attention"] / (attn_ms * 1e-3) / 1e9
+    seq_steps = W.num_seqs * world / (ms * 1e-3)
+    traffic = recorded_traffic(W)
+    line = {
+        "metric": METRIC,
+        "value": round(gbs, 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": wl.DTYPE_NAMES[W.kv_dtype],
+        "data": "synthetic (seeded N(0,1) q/K/V, seeded block tables)",
+        "seq_steps_per_s_per_layer": round(seq_steps, 1),
+        "pct_of_hbm_peak": round(100 * gbs / peak, 2),
+        "config": {
+            "workload": workload_name(W),
+            "batch": W.num_seqs, "total_q": W.total_q, "q_heads": W.num_q_heads,
+            "kv_heads": W.num_kv_heads, "head_dim": W.head_dim, "block_size": W.block_size,
+            "num_blocks": W.num_blocks, "mean_context": round(float(W.seqlens_k.mean()), 1),
+            "max_context": W.max_context_len, "partition_size": W.partition_size or "auto",
+            "kv_bytes_per_step": by["kv"],
+            "l2": "inputs larger than L2 (KV read per step >> 126 MB); no flush",
+            "parallelism": f"replicas x{world}",
+        },
+        "roofline": {
+            "bound": "hbm", "kernel": "pa_decode" if W.decode else "pa_varlen",
+            "achieved": round(attn_gbs, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(attn_gbs / peak, 4), "traffic": traffic,
+            "peak_source": f"{peak_kind} hbm_gbs", "attention_ms": round(attn_ms, 5),
+            "algorithmic_bytes": by["attention"],
+        },
+        "clocks": clocks.summary(),
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    if e2e:
+        e2e_ms, h2d, d2h = e2e
+        line["e2e"] = {"value": round(by["kv"] * world / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                       "ms_per_step": round(e2e_ms, 5)}
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(W, budget_s=12.0)
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def recorded_traffic(W):
+    """DRAM bytes per attention launch from the committed ncu summary, if it
+    was taken on this workload with the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
+        return None
+    key = W.name
+    entry = rec.get(key)
+    if not entry or entry.get("kernel_sha") != kernel_sha():
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
+def kernel_sha():
+    import hashlib
+    h = hashlib.sha256()
+    for name in ("paged_attention.cu", "pa_device.cuh", "pa_launch.h"):
+        with open(os.path.join(ROOT, "paged_kv_cache_lens_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+# --------------------------------------------------------------------------
+# CPU oracle (baseline leg and the reference arm)
+# --------------------------------------------------------------------------
+
+def _oracle_sample(W, n_seqs, threads):
+    """Run the oracle's step (cache write of the new rows + attention) over the
+    first n_seqs requests; returns (seconds, kv bytes processed, requests)."""
+    from oracle import pa_oracle
+    rows = list(range(int(W.cu_seqlens_q[n_seqs])))
+    reqs = n_seqs
+    blocks = set()
+    for r in range(reqs):
+        n = -(-int(W.seqlens_k[r]) // W.block_size)
+        blocks.update(int(b) for b in W.block_tables[r, :n])
+    blocks = np.array(sorted(blocks), np.int64)
+    shape = (W.num_blocks, W.num_kv_heads, W.block_size, W.head_dim)
+    dt = np.uint8 if W.kv_dtype == wl.FP8_E4M3 else np.uint16
+    kc, vc = np.empty(shape, dt), np.empty(shape, dt)
+    keep = np.isin(W.prefill_slots // W.block_size, blocks)
+    pa_oracle.reshape_and_cache(W.prefill_k[keep], W.prefill_v[keep], W.src_dtype,
+                                W.prefill_slots[keep], kc, vc, W.block_size, W.kv_dtype,
+                                W.k_scale, W.v_scale)
+    nrows = len(rows)
+    t = time.perf_counter()
+    pa_oracle.reshape_and_cache(W.new_k[:nrows], W.new_v[:nrows], W.src_dtype,
+                                W.new_slots[:nrows], kc, vc, W.block_size, W.kv_dtype,
+                                W.k_scale, W.v_scale)
+    cu = W.cu_seqlens_q[:reqs + 1]
+    pa_oracle.paged_attention(W.q[:nrows], W.q_dtype, cu, W.seqlens_k[:reqs], kc, vc, W.kv_dtype,
+                              W.block_tables[:reqs], W.scale, W.k_scale, W.v_scale,
+                              num_threads=threads)
+    dt_s = time.perf_counter() - t
+    per_tok = 2 * W.num_kv_heads * W.head_dim * W.kv_elem_bytes()
+    return dt_s, int(W.seqlens_k[:reqs].astype(np.int64).sum()) * per_tok, reqs
+
+
+def cpu_baseline(W, budget_s=12.0):
+    threads = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    n = 1
+    t, b, reqs = _oracle_sample(W, n, threads)
+    # grow the sample to roughly the time budget (bounded by the batch)
+    if t < budget_s and n < W.num_seqs:
+        n = int(min(W.num_seqs, max(2, budget_s / max(t, 1e-3))))
+        t, b, reqs = _oracle_sample(W, n, threads)
+    return {"value": round(b / t / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"{reqs} of {W.num_seqs} requests of the step (cache write + attention, "
+                      f"fp64), {t:.1f} s", "seq_steps_per_s_per_layer": round(reqs / t, 3)}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    W = wl.config(args.workload)
+    threads = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    # size one step's sample so that warmup + steps stay within a few minutes
+    t1, _, _ = _oracle_sample(W, 1, threads)
+    n = int(min(W.num_seqs, max(1, 3.0 / max(t1, 1e-3))))
+    times, bytes_, reqs = [], 0, n
+    for i in range(args.warmup + args.steps):
+        t, b, reqs = _oracle_sample(W, n, threads)
+        if i >= args.warmup:
+            times.append(t)
+            bytes_ = b
+    s = float(np.mean(times)) if times else float("nan")
+    value = bytes_ / s / 1e9
+    line = {
+        "metric": METRIC, "impl": "reference", "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(s * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_name(W), "batch": W.num_seqs,
+                   "sample_requests_per_step": reqs},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": threads,
+                         "kind": "oracle",
+                         "sample": f"{reqs} of {W.num_seqs} requests per step (fp64 oracle)"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_native(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,201 @@
+/*
+ * libpa — paged KV-cache attention for NVIDIA B200 (sm_100a).
+ *
+ * A block-paged KV cache ("PagedAttention 与 Continuous Batching", §3.2-§3.3:
+ * fixed 16-token physical blocks, one block table per request mapping logical
+ * to physical blocks) and the three data-parallel steps that touch it:
+ *
+ *   pa_reshape_and_cache  write this step's new K/V rows into their physical
+ *                         slots (§3.3 decode steps 1-2; slot_mapping from §2.5
+ *                         step 4).
+ *   pa_decode             one query row per sequence attends its cached
+ *                         context through the block table (§3.6 PagedAttention
+ *                         Kernel), query heads of a GQA group sharing each KV
+ *                         block, long contexts split into partitions merged by
+ *                         a log-sum-exp reduce.
+ *   pa_varlen             the packed mixed prefill/decode step: query rows of
+ *                         all scheduled requests packed as [total_q, H, D],
+ *                         cu_seqlens marking request boundaries ("推理优化与服务：
+ *                         从 PagedAttention 到分离式部署", 最新进展 on the V1
+ *                         unified step), causal within each request.
+ *
+ * Conventions for every entry point:
+ *   - Pointers named as device pointers are CUDA device memory owned by the
+ *     caller; the library allocates nothing, keeps no state between calls
+ *     (apart from one device error word, see pa_device_error) and never
+ *     synchronises the stream.  Work is enqueued on `stream` (a cudaStream_t;
+ *     NULL is the legacy default stream) and the call returns.
+ *   - Arguments are validated on the host before anything is enqueued; a
+ *     failed check returns PA_ERR_INVALID_ARG / PA_ERR_UNSUPPORTED /
+ *     PA_ERR_WORKSPACE and enqueues nothing.  A failed launch returns
+ *     PA_ERR_CUDA.  No exception crosses this interface.
+ *   - KV pool layout (a reading: the pages fix no axis order): k_cache and
+ *     v_cache are [num_blocks][num_kv_heads][block_size][head_dim], row-major,
+ *     so each (block, head) tile is one contiguous run.  Token t of a request
+ *     with block table bt lives at slot bt[t / block_size] * block_size +
+ *     t % block_size.
+ *   - Block-table entries at or past ceil(len / block_size) are never read.
+ *     Entries that are read and fall outside [0, num_blocks) are skipped
+ *     (treated as masked) and recorded in the device error word.
+ *   - GQA: query head hq reads KV head hq / (num_q_heads / num_kv_heads).
+ *   - Attention accumulates in fp32; softmax is exact up to rounding.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PA_F16 = 0,        /* IEEE binary16 */
+    PA_BF16 = 1,       /* bfloat16 */
+    PA_FP8_E4M3 = 2,   /* OCP FP8 E4M3 (KV pool only), with per-head fp32 scales */
+    PA_F32 = 3         /* IEEE binary32 (outputs only) */
+} pa_dtype;
+
+typedef enum {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned buffer */
+    PA_ERR_UNSUPPORTED = 2,   /* dtype / head_dim / block_size / group size not built */
+    PA_ERR_WORKSPACE = 3,     /* workspace smaller than the *_workspace_size figure */
+    PA_ERR_OUT_OF_RANGE = 4,  /* a kernel met a block id or slot outside the pool */
+    PA_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed */
+    PA_ERR_TIMEOUT = 6        /* a kernel's bounded wait for its own copies expired */
+} pa_status;
+
+/* Description of one layer's KV pool (a host struct; the scale pointers in it
+ * are device pointers). */
+typedef struct {
+    int32_t num_blocks;     /* physical blocks in the pool */
+    int32_t block_size;     /* tokens per block: 16 */
+    int32_t num_kv_heads;
+    int32_t head_dim;       /* 64, 128 or 256 (FP8: 128 or 256) */
+    pa_dtype kv_dtype;      /* PA_F16, PA_BF16 or PA_FP8_E4M3 */
+    const float* k_scale;   /* [num_kv_heads] device fp32, FP8 only, else NULL */
+    const float* v_scale;   /* [num_kv_heads] device fp32, FP8 only, else NULL */
+} pa_cache_desc;
+
+/*
+ * Human-readable name of a status code (static storage, never NULL).
+ */
+const char* pa_status_string(pa_status status);
+
+/*
+ * Write new K/V rows into the paged pool ("PagedAttention 与 Continuous
+ * Batching", §3.3: append each new token's K/V into the last block if it has
+ * room, else into a freshly allocated block; the scheduler encodes the chosen
+ * slot per token in slot_mapping, §2.5 step 4).
+ *
+ * key, value   : device, num_tokens rows; row i starts at element
+ *                i * token_stride and holds [num_kv_heads][head_dim]
+ *                contiguous elements of src_dtype (PA_F16 or PA_BF16).
+ *                token_stride >= num_kv_heads * head_dim lets K/V sit inside
+ *                a fused QKV buffer.  Both must be 16-byte aligned, and
+ *                token_stride * element size a multiple of 16 bytes.
+ * slot_mapping : device int64 [num_tokens]; slot = block * block_size +
+ *                offset; a negative slot skips the token (padding).  Slots
+ *                must be unique within one call (duplicates race).
+ * k_cache, v_cache : device pools (layout above), written in place.
+ * cache        : pool description.  kv_dtype == src_dtype copies the bits;
+ *                PA_FP8_E4M3 stores e4m3(round-to-nearest-even, saturating)
+ *                of x / k_scale[h] (resp. v_scale[h]), the quotient taken as
+ *                an IEEE fp32 division.
+ * A slot beyond the pool is skipped and recorded in the device error word.
+ */
+pa_status pa_reshape_and_cache(const void* key, const void* value, pa_dtype src_dtype,
+                               int64_t num_tokens, int64_t token_stride,
+                               const int64_t* slot_mapping, void* k_cache, void* v_cache,
+                               const pa_cache_desc* cache, void* stream);
+
+/*
+ * Bytes of workspace pa_decode needs for these sizes (0 when no sequence can
+ * span more than one partition).  partition_size as passed to pa_decode
+ * (0 = automatic, which is what this function then assumes).
+ */
+size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t head_dim,
+                                int32_t max_context_len, int32_t partition_size);
+
+/*
+ * Paged decode attention ("PagedAttention 与 Continuous Batching", §3.6): for
+ * every sequence b and query head hq,
+ *   out[b][hq] = sum_t softmax_t(scale * <q[b][hq], K_t>) V_t
+ * over the context_lens[b] cached tokens of sequence b (the current token's
+ * K/V already written by pa_reshape_and_cache), K_t/V_t fetched through
+ * block_tables[b].  A sequence with context_lens[b] == 0 yields zeros.
+ *
+ * out          : device [batch][num_q_heads][head_dim] of out_dtype
+ *                (PA_F16, PA_BF16 or PA_F32; rounded to nearest even).
+ * q            : device [batch][num_q_heads][head_dim] of q_dtype.  With a
+ *                16-bit pool q_dtype must equal the pool dtype; with an FP8
+ *                pool it may be PA_BF16 or PA_F16 (|q| must stay below 65504,
+ *                the products being taken in f16).
+ * block_tables : device int32 [batch][max_blocks_per_seq].
+ * context_lens : device int32 [batch], each in [0, max_context_len].
+ * max_context_len: host upper bound of context_lens, used to size the grid
+ *                and the workspace without reading device memory.
+ * partition_size: tokens per split-K partition (a multiple of 64, or 0 for
+ *                an automatic choice).  Sequences longer than one partition
+ *                are split; partial results (running max, sum and
+ *                unnormalised output per partition) are merged with the
+ *                log-sum-exp rule in a second pass.
+ * workspace    : device scratch of at least pa_decode_workspace_size(...)
+ *                bytes, 256-byte aligned, contents irrelevant on entry.
+ *                Concurrent calls must not share a workspace.
+ */
+pa_status pa_decode(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dtype,
+                    int32_t batch, int32_t num_q_heads, const void* k_cache,
+                    const void* v_cache, const pa_cache_desc* cache,
+                    const int32_t* block_tables, int32_t max_blocks_per_seq,
+                    const int32_t* context_lens, int32_t max_context_len, float scale,
+                    int32_t partition_size, void* workspace, size_t workspace_bytes,
+                    void* stream);
+
+/*
+ * Bytes of workspace pa_varlen needs for these sizes.
+ */
+size_t pa_varlen_workspace_size(int32_t num_seqs, int32_t total_q, int32_t num_q_heads,
+                                int32_t head_dim, int32_t max_context_len);
+
+/*
+ * Packed mixed prefill/decode attention.  Request r owns query rows
+ * cu_seqlens_q[r] .. cu_seqlens_q[r+1]-1 (q_len_r rows) and seqlens_k[r] keys
+ * (kv_len_r = cached + this step's new tokens, the new ones already written by
+ * pa_reshape_and_cache).  Row i of request r sits at absolute position
+ * kv_len_r - q_len_r + i and attends keys 0 .. kv_len_r - q_len_r + i
+ * (causal mask aligned to the bottom right).  Rows with no visible key yield
+ * zeros.  q_len 1 rows are decode rows; longer ones are prefill chunks.
+ *
+ * out, q       : device [total_q][num_q_heads][head_dim].
+ * cu_seqlens_q : device int32 [num_seqs + 1], non-decreasing, cu[0] = 0,
+ *                cu[num_seqs] = total_q.
+ * seqlens_k    : device int32 [num_seqs], kv_len_r >= q_len_r.
+ * max_q_len, max_context_len: host upper bounds of q_len_r and kv_len_r.
+ * block_tables : device int32 [num_seqs][max_blocks_per_seq].
+ * workspace    : device scratch of at least pa_varlen_workspace_size(...)
+ *                bytes, 256-byte aligned.
+ */
+pa_status pa_varlen(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dtype,
+                    int32_t total_q, int32_t num_seqs, int32_t num_q_heads,
+                    const int32_t* cu_seqlens_q, const int32_t* seqlens_k, int32_t max_q_len,
+                    int32_t max_context_len, const void* k_cache, const void* v_cache,
+                    const pa_cache_desc* cache, const int32_t* block_tables,
+                    int32_t max_blocks_per_seq, float scale, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/*
+ * Read and clear the device error word that kernels set when they skip an
+ * out-of-range block id or slot (PA_ERR_OUT_OF_RANGE) or give up a bounded
+ * wait (PA_ERR_TIMEOUT).  Synchronises `stream` first.  Returns PA_OK when no
+ * kernel reported anything since the last call.
+ */
+pa_status pa_device_error(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

@@ -1,0 +1,330 @@
+// C ABI of libpa: argument validation, workspace sizing, tensor-map set-up and
+// dispatch to the kernels.  See include/pa.h for the contract of every call.
+#include "pa.h"
+#include "pa_launch.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cstdint>
+#include <cstring>
+
+namespace pa {
+
+namespace {
+
+constexpr int kBlockSize = 16;
+constexpr int64_t kAlign = 256;
+
+inline int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+inline bool aligned(const void* p, uintptr_t a) {
+  return (reinterpret_cast<uintptr_t>(p) % a) == 0;
+}
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Automatic partition size: 512 tokens, halved (down to 128) while the
+// launch would have fewer than ~2048 (row, head, partition) items, so short
+// batches of long contexts still fill the 148 SMs.
+int32_t auto_partition(int64_t rows, int32_t num_q_heads, int32_t max_context_len) {
+  int32_t ps = 512;
+  while (ps > 128 && rows * num_q_heads * cdiv(max_context_len, ps) < 2048) ps /= 2;
+  return ps;
+}
+
+int32_t resolve_partition(int64_t rows, int32_t num_q_heads, int32_t max_context_len,
+                          int32_t requested) {
+  return requested > 0 ? requested : auto_partition(rows, num_q_heads, max_context_len);
+}
+
+bool valid_partition(int32_t ps) { return ps == 0 || (ps >= 64 && ps <= 1024 && ps % 64 == 0); }
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+size_t elem_size(pa_dtype t) {
+  switch (t) {
+    case PA_F16: case PA_BF16: return 2;
+    case PA_FP8_E4M3: return 1;
+    case PA_F32: return 4;
+  }
+  return 0;
+}
+
+pa_status check_cache(const pa_cache_desc* c) {
+  if (!c) return PA_ERR_INVALID_ARG;
+  if (c->num_blocks <= 0 || c->num_kv_heads <= 0 || c->head_dim <= 0) return PA_ERR_INVALID_ARG;
+  if (c->block_size != kBlockSize) return PA_ERR_UNSUPPORTED;
+  if (c->kv_dtype != PA_F16 && c->kv_dtype != PA_BF16 && c->kv_dtype != PA_FP8_E4M3)
+    return PA_ERR_UNSUPPORTED;
+  if (c->kv_dtype == PA_FP8_E4M3 && (!c->k_scale || !c->v_scale)) return PA_ERR_INVALID_ARG;
+  // TMA row coordinates are 32-bit
+  if (static_cast<int64_t>(c->num_blocks) * c->num_kv_heads * kBlockSize > INT_MAX)
+    return PA_ERR_UNSUPPORTED;
+  return PA_OK;
+}
+
+}  // namespace
+
+DecodeWorkspace decode_workspace_layout(int64_t rows, int32_t num_q_heads, int32_t head_dim,
+                                        int32_t max_parts) {
+  DecodeWorkspace w{0, 0, 0, 0};
+  if (max_parts <= 1) return w;
+  const int64_t n = rows * num_q_heads * max_parts;
+  w.m_off = 0;
+  w.l_off = align_up(n * 4, kAlign);
+  w.o_off = w.l_off + align_up(n * 4, kAlign);
+  w.total = w.o_off + align_up(n * head_dim * 4, kAlign);
+  return w;
+}
+
+bool make_pool_tensor_map(CUtensorMap* map, const void* base, int kv_dtype, int64_t rows,
+                          int32_t head_dim, int32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const int esz = (kv_dtype == PA_FP8_E4M3) ? 1 : 2;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(head_dim) * esz};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esz), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, esz == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16,
+                   2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" {
+
+const char* pa_status_string(pa_status status) {
+  switch (status) {
+    case PA_OK: return "PA_OK";
+    case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG: invalid argument";
+    case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED: configuration not supported";
+    case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE: workspace too small";
+    case PA_ERR_OUT_OF_RANGE: return "PA_ERR_OUT_OF_RANGE: block id or slot outside the pool";
+    case PA_ERR_CUDA: return "PA_ERR_CUDA: CUDA runtime or launch failure";
+    case PA_ERR_TIMEOUT: return "PA_ERR_TIMEOUT: a kernel gave up a bounded wait";
+  }
+  return "PA_ERR_UNKNOWN";
+}
+
+pa_status pa_reshape_and_cache(const void* key, const void* value, pa_dtype src_dtype,
+                               int64_t num_tokens, int64_t token_stride,
+                               const int64_t* slot_mapping, void* k_cache, void* v_cache,
+                               const pa_cache_desc* cache, void* stream) {
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (num_tokens < 0) return PA_ERR_INVALID_ARG;
+  if (num_tokens == 0) return PA_OK;
+  if (!key || !value || !slot_mapping || !k_cache || !v_cache) return PA_ERR_INVALID_ARG;
+  if (src_dtype != PA_F16 && src_dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if (cache->kv_dtype != PA_FP8_E4M3 && cache->kv_dtype != src_dtype) return PA_ERR_UNSUPPORTED;
+  if (cache->head_dim % 8 != 0) return PA_ERR_UNSUPPORTED;
+  const int64_t row = static_cast<int64_t>(cache->num_kv_heads) * cache->head_dim;
+  if (token_stride < row) return PA_ERR_INVALID_ARG;
+  if ((token_stride * 2) % 16 != 0) return PA_ERR_INVALID_ARG;
+  const uintptr_t pool_align = cache->kv_dtype == PA_FP8_E4M3 ? 8 : 16;
+  if (!aligned(key, 16) || !aligned(value, 16) || !aligned(k_cache, pool_align) ||
+      !aligned(v_cache, pool_align) || !aligned(slot_mapping, 8))
+    return PA_ERR_INVALID_ARG;
+  cudaError_t e = launch_reshape_and_cache(
+      key, value, src_dtype, num_tokens, token_stride, slot_mapping, k_cache, v_cache,
+      cache->num_blocks, cache->block_size, cache->num_kv_heads, cache->head_dim,
+      cache->kv_dtype, cache->k_scale, cache->v_scale, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t head_dim,
+                                int32_t max_context_len, int32_t partition_size) {
+  if (batch <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_context_len <= 0) return 0;
+  if (!valid_partition(partition_size)) return 0;
+  const int32_t ps = resolve_partition(batch, num_q_heads, max_context_len, partition_size);
+  const int32_t parts = static_cast<int32_t>(cdiv(max_context_len, ps));
+  return decode_workspace_layout(batch, num_q_heads, head_dim, parts).total;
+}
+
+size_t pa_varlen_workspace_size(int32_t num_seqs, int32_t total_q, int32_t num_q_heads,
+                                int32_t head_dim, int32_t max_context_len) {
+  if (num_seqs <= 0 || total_q <= 0 || num_q_heads <= 0 || head_dim <= 0) return 0;
+  const int64_t maps = 2 * align_up(static_cast<int64_t>(total_q) * 4, kAlign);
+  if (max_context_len <= 0) return static_cast<size_t>(maps);
+  const int32_t ps = auto_partition(total_q, num_q_heads, max_context_len);
+  const int32_t parts = static_cast<int32_t>(cdiv(max_context_len, ps));
+  return static_cast<size_t>(maps) +
+         decode_workspace_layout(total_q, num_q_heads, head_dim, parts).total;
+}
+
+static pa_status check_attention(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dtype,
+                                 int32_t num_q_heads, const void* k_cache, const void* v_cache,
+                                 const pa_cache_desc* cache, const int32_t* block_tables,
+                                 int32_t max_blocks_per_seq, int32_t max_context_len) {
+  pa_status st = check_cache(cache);
+  if (st != PA_OK) return st;
+  if (!out || !q || !k_cache || !v_cache || !block_tables) return PA_ERR_INVALID_ARG;
+  if (num_q_heads <= 0 || num_q_heads % cache->num_kv_heads != 0) return PA_ERR_INVALID_ARG;
+  if (max_context_len < 0 || max_blocks_per_seq < 0) return PA_ERR_INVALID_ARG;
+  if (cdiv(max_context_len, kBlockSize) > max_blocks_per_seq) return PA_ERR_INVALID_ARG;
+  if (out_dtype != PA_F16 && out_dtype != PA_BF16 && out_dtype != PA_F32)
+    return PA_ERR_UNSUPPORTED;
+  const int32_t group = num_q_heads / cache->num_kv_heads;
+  if (!attention_supported(q_dtype, cache->kv_dtype, cache->head_dim, group))
+    return PA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(out, elem_size(out_dtype)) || !aligned(block_tables, 4))
+    return PA_ERR_INVALID_ARG;
+  return PA_OK;
+}
+
+static pa_status run_attention(AttnArgs& a, const pa_cache_desc* cache, int32_t max_context_len,
+                               int32_t ps, float* ws_base, size_t ws_bytes, size_t ws_needed,
+                               cudaStream_t stream) {
+  a.partition_size = ps;
+  a.max_context_len = max_context_len;
+  a.max_parts = static_cast<int32_t>(cdiv(max_context_len > 0 ? max_context_len : 1, ps));
+  if (a.max_parts > 1) {
+    if (!ws_base || ws_bytes < ws_needed) return PA_ERR_WORKSPACE;
+    if (!aligned(ws_base, 256)) return PA_ERR_INVALID_ARG;
+    DecodeWorkspace w = decode_workspace_layout(a.rows, a.num_q_heads, a.head_dim, a.max_parts);
+    auto* b = reinterpret_cast<uint8_t*>(ws_base);
+    a.ws_m = reinterpret_cast<float*>(b + w.m_off);
+    a.ws_l = reinterpret_cast<float*>(b + w.l_off);
+    a.ws_o = reinterpret_cast<float*>(b + w.o_off);
+  } else {
+    a.ws_m = a.ws_l = a.ws_o = nullptr;
+  }
+  const int64_t pool_rows = static_cast<int64_t>(cache->num_blocks) * cache->num_kv_heads *
+                            kBlockSize;
+  CUtensorMap kmap, vmap;
+  if (!make_pool_tensor_map(&kmap, a.k_cache, cache->kv_dtype, pool_rows, cache->head_dim,
+                            kBlockSize) ||
+      !make_pool_tensor_map(&vmap, a.v_cache, cache->kv_dtype, pool_rows, cache->head_dim,
+                            kBlockSize))
+    return PA_ERR_CUDA;
+  cudaError_t e = launch_paged_attention(a, kmap, vmap, stream);
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+}
+
+static void fill_common(AttnArgs& a, void* out, pa_dtype out_dtype, const void* q,
+                        pa_dtype q_dtype, int32_t num_q_heads, const void* k_cache,
+                        const void* v_cache, const pa_cache_desc* cache,
+                        const int32_t* block_tables, int32_t max_blocks_per_seq, float scale) {
+  std::memset(&a, 0, sizeof(a));
+  a.out = out;
+  a.q = q;
+  a.out_dtype = out_dtype;
+  a.q_dtype = q_dtype;
+  a.kv_dtype = cache->kv_dtype;
+  a.num_q_heads = num_q_heads;
+  a.num_kv_heads = cache->num_kv_heads;
+  a.head_dim = cache->head_dim;
+  a.group = num_q_heads / cache->num_kv_heads;
+  a.num_blocks = cache->num_blocks;
+  a.block_size = cache->block_size;
+  a.block_tables = block_tables;
+  a.max_blocks_per_seq = max_blocks_per_seq;
+  a.k_scale = cache->k_scale;
+  a.v_scale = cache->v_scale;
+  a.scale = scale;
+  a.k_cache = k_cache;
+  a.v_cache = v_cache;
+}
+
+pa_status pa_decode(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dtype,
+                    int32_t batch, int32_t num_q_heads, const void* k_cache,
+                    const void* v_cache, const pa_cache_desc* cache,
+                    const int32_t* block_tables, int32_t max_blocks_per_seq,
+                    const int32_t* context_lens, int32_t max_context_len, float scale,
+                    int32_t partition_size, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  if (batch < 0) return PA_ERR_INVALID_ARG;
+  pa_status st = check_attention(out, out_dtype, q, q_dtype, num_q_heads, k_cache, v_cache,
+                                 cache, block_tables, max_blocks_per_seq, max_context_len);
+  if (st != PA_OK) return st;
+  if (!context_lens) return PA_ERR_INVALID_ARG;
+  if (!valid_partition(partition_size)) return PA_ERR_INVALID_ARG;
+  if (batch == 0) return PA_OK;
+  AttnArgs a;
+  fill_common(a, out, out_dtype, q, q_dtype, num_q_heads, k_cache, v_cache, cache, block_tables,
+              max_blocks_per_seq, scale);
+  a.rows = batch;
+  a.num_seqs = batch;
+  a.context_lens = context_lens;
+  const int32_t ps = resolve_partition(batch, num_q_heads, max_context_len, partition_size);
+  const size_t need =
+      pa_decode_workspace_size(batch, num_q_heads, cache->head_dim, max_context_len, ps);
+  return run_attention(a, cache, max_context_len, ps, static_cast<float*>(workspace),
+                       workspace_bytes, need, static_cast<cudaStream_t>(stream));
+}
+
+pa_status pa_varlen(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dtype,
+                    int32_t total_q, int32_t num_seqs, int32_t num_q_heads,
+                    const int32_t* cu_seqlens_q, const int32_t* seqlens_k, int32_t max_q_len,
+                    int32_t max_context_len, const void* k_cache, const void* v_cache,
+                    const pa_cache_desc* cache, const int32_t* block_tables,
+                    int32_t max_blocks_per_seq, float scale, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  if (total_q < 0 || num_seqs < 0 || max_q_len < 0) return PA_ERR_INVALID_ARG;
+  pa_status st = check_attention(out, out_dtype, q, q_dtype, num_q_heads, k_cache, v_cache,
+                                 cache, block_tables, max_blocks_per_seq, max_context_len);
+  if (st != PA_OK) return st;
+  if (!cu_seqlens_q || !seqlens_k) return PA_ERR_INVALID_ARG;
+  if (max_q_len > max_context_len) return PA_ERR_INVALID_ARG;
+  if (total_q == 0) return PA_OK;
+  if (num_seqs == 0) return PA_ERR_INVALID_ARG;
+  const size_t need = pa_varlen_workspace_size(num_seqs, total_q, num_q_heads, cache->head_dim,
+                                               max_context_len);
+  if (!workspace || workspace_bytes < need) return PA_ERR_WORKSPACE;
+  if (!aligned(workspace, 256)) return PA_ERR_INVALID_ARG;
+  auto* b = static_cast<uint8_t*>(workspace);
+  const int64_t map_bytes = align_up(static_cast<int64_t>(total_q) * 4, kAlign);
+  int32_t* row_seq = reinterpret_cast<int32_t*>(b);
+  int32_t* row_len = reinterpret_cast<int32_t*>(b + map_bytes);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (launch_varlen_prep(total_q, num_seqs, cu_seqlens_q, seqlens_k, row_seq, row_len, s) !=
+      cudaSuccess)
+    return PA_ERR_CUDA;
+  AttnArgs a;
+  fill_common(a, out, out_dtype, q, q_dtype, num_q_heads, k_cache, v_cache, cache, block_tables,
+              max_blocks_per_seq, scale);
+  a.rows = total_q;
+  a.num_seqs = num_seqs;
+  a.row_seq = row_seq;
+  a.row_len = row_len;
+  a.cu_seqlens_q = cu_seqlens_q;
+  a.seqlens_k = seqlens_k;
+  const int32_t ps = auto_partition(total_q, num_q_heads, max_context_len);
+  return run_attention(a, cache, max_context_len, ps,
+                       reinterpret_cast<float*>(b + 2 * map_bytes),
+                       workspace_bytes - 2 * map_bytes, need - 2 * map_bytes, s);
+}
+
+pa_status pa_device_error(void* stream) {
+  cudaError_t e;
+  unsigned v = read_and_clear_error_word(static_cast<cudaStream_t>(stream), &e);
+  if (e != cudaSuccess) return PA_ERR_CUDA;
+  if (v == kErrTimeout) return PA_ERR_TIMEOUT;
+  if (v != 0) return PA_ERR_OUT_OF_RANGE;
+  return PA_OK;
+}
+
+}  // extern "C"

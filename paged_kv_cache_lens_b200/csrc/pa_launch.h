@@ -1,0 +1,74 @@
+// Host-side launch descriptors shared by the C-ABI layer and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace pa {
+
+// Device error word codes (the first one reported wins until the host clears it).
+enum : unsigned { kErrNone = 0, kErrBlockRange = 1, kErrSlotRange = 2, kErrTimeout = 3 };
+
+// Everything one attention launch needs; plain pointers and sizes.
+struct AttnArgs {
+  void* out;                    // [rows][Hq][D]
+  const void* q;                // [rows][Hq][D]
+  int out_dtype, q_dtype, kv_dtype;
+  int32_t rows;                 // query rows (sequences for decode, total_q for varlen)
+  int32_t num_q_heads, num_kv_heads, head_dim, group;
+  int32_t num_blocks, block_size;
+  const int32_t* block_tables;  // [num_seqs][max_blocks_per_seq]
+  int32_t max_blocks_per_seq;
+  const int32_t* context_lens;  // decode: [rows]; varlen: nullptr
+  const int32_t* row_seq;       // varlen: request of each row (workspace)
+  const int32_t* row_len;       // varlen: visible keys of each row (workspace)
+  const int32_t* cu_seqlens_q;  // varlen only
+  const int32_t* seqlens_k;     // varlen only
+  int32_t num_seqs;
+  const float* k_scale;
+  const float* v_scale;
+  float scale;
+  int32_t max_context_len;      // host bound; longer rows are clamped to it
+  int32_t partition_size;       // tokens per split-K partition
+  int32_t max_parts;            // partitions of the longest row
+  float* ws_m;                  // [rows][Hq][max_parts] running max (log2 domain)
+  float* ws_l;                  // [rows][Hq][max_parts] running sum
+  float* ws_o;                  // [rows][Hq][max_parts][D] unnormalised output
+  const void* k_cache;
+  const void* v_cache;
+};
+
+// Workspace carve-up (all offsets 256-byte aligned).
+struct DecodeWorkspace {
+  size_t m_off, l_off, o_off, total;
+};
+
+DecodeWorkspace decode_workspace_layout(int64_t rows, int32_t num_q_heads, int32_t head_dim,
+                                        int32_t max_parts);
+
+// Tensor maps over the pool viewed as [num_blocks*Hkv*block_size rows, D cols]
+// with 128-byte boxes and the 128-byte swizzle.  Returns false on failure.
+bool make_pool_tensor_map(CUtensorMap* map, const void* base, int kv_dtype, int64_t rows,
+                          int32_t head_dim, int32_t box_rows);
+
+cudaError_t launch_paged_attention(const AttnArgs& a, const CUtensorMap& kmap,
+                                   const CUtensorMap& vmap, cudaStream_t stream);
+
+cudaError_t launch_varlen_prep(int32_t total_q, int32_t num_seqs, const int32_t* cu_seqlens_q,
+                               const int32_t* seqlens_k, int32_t* row_seq, int32_t* row_len,
+                               cudaStream_t stream);
+
+cudaError_t launch_reshape_and_cache(const void* key, const void* value, int src_dtype,
+                                     int64_t num_tokens, int64_t token_stride,
+                                     const int64_t* slot_mapping, void* k_cache, void* v_cache,
+                                     int32_t num_blocks, int32_t block_size, int32_t num_kv_heads,
+                                     int32_t head_dim, int kv_dtype, const float* k_scale,
+                                     const float* v_scale, cudaStream_t stream);
+
+bool attention_supported(int q_dtype, int kv_dtype, int32_t head_dim, int32_t group);
+
+unsigned int read_and_clear_error_word(cudaStream_t stream, cudaError_t* err);
+
+}  // namespace pa

@@ -1,0 +1,210 @@
+"""Python binding of libpa (ctypes): argument marshalling only.
+
+Every function here has the name of the C entry point it calls and does no
+arithmetic of its own: it turns torch tensors into device pointers, sizes and
+dtype codes, passes the current CUDA stream, and raises :class:`PaError` on a
+non-zero status.  The library must be built in-tree
+(``python -m paged_kv_cache_lens_b200.build``); importing this module without
+it raises, so there is no silent CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpa.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "pa.h")
+
+PA_F16, PA_BF16, PA_FP8_E4M3, PA_F32 = 0, 1, 2, 3
+PA_OK = 0
+STATUS_NAMES = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED",
+                3: "PA_ERR_WORKSPACE", 4: "PA_ERR_OUT_OF_RANGE", 5: "PA_ERR_CUDA",
+                6: "PA_ERR_TIMEOUT"}
+BLOCK_SIZE = 16
+
+
+class PaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {pa_status_string(status)}")
+
+
+class pa_cache_desc(ctypes.Structure):
+    _fields_ = [("num_blocks", ctypes.c_int32), ("block_size", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("kv_dtype", ctypes.c_int), ("k_scale", ctypes.c_void_p),
+                ("v_scale", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libpa.so and declare its signatures.  Raises if it is missing."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is not built; run `python -m paged_kv_cache_lens_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    E, F = ctypes.c_int, ctypes.c_float
+    D = ctypes.POINTER(pa_cache_desc)
+    lib.pa_status_string.argtypes = [E]
+    lib.pa_status_string.restype = ctypes.c_char_p
+    lib.pa_reshape_and_cache.argtypes = [P, P, E, i64, i64, P, P, P, D, P]
+    lib.pa_reshape_and_cache.restype = E
+    lib.pa_decode_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+    lib.pa_decode_workspace_size.restype = sz
+    lib.pa_decode.argtypes = [P, E, P, E, i32, i32, P, P, D, P, i32, P, i32, F, i32, P, sz, P]
+    lib.pa_decode.restype = E
+    lib.pa_varlen_workspace_size.argtypes = [i32, i32, i32, i32, i32]
+    lib.pa_varlen_workspace_size.restype = sz
+    lib.pa_varlen.argtypes = [P, E, P, E, i32, i32, i32, P, P, i32, i32, P, P, D, P, i32, F, P,
+                              sz, P]
+    lib.pa_varlen.restype = E
+    lib.pa_device_error.argtypes = [P]
+    lib.pa_device_error.restype = E
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def declared_functions(header: str = HEADER):
+    """Names of the entry points include/pa.h declares."""
+    text = open(header).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text)))
+
+
+# --------------------------------------------------------------------------
+# marshalling helpers
+# --------------------------------------------------------------------------
+
+def dtype_code(t: torch.dtype, fp8_if_byte: bool = False) -> int:
+    if t == torch.float16:
+        return PA_F16
+    if t == torch.bfloat16:
+        return PA_BF16
+    if t == torch.float32:
+        return PA_F32
+    if t in (torch.uint8, getattr(torch, "float8_e4m3fn", None)):
+        return PA_FP8_E4M3
+    raise ValueError(f"no libpa dtype for {t}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def cache_desc(k_cache: torch.Tensor, k_scale=None, v_scale=None) -> pa_cache_desc:
+    nb, hkv, bs, d = k_cache.shape
+    return pa_cache_desc(nb, bs, hkv, d, dtype_code(k_cache.dtype), _ptr(k_scale).value
+                         if k_scale is not None else None,
+                         _ptr(v_scale).value if v_scale is not None else None)
+
+
+def _check(status: int, where: str):
+    if status != PA_OK:
+        raise PaError(status, where)
+
+
+# --------------------------------------------------------------------------
+# entry points
+# --------------------------------------------------------------------------
+
+def pa_status_string(status: int) -> str:
+    try:
+        return load_library().pa_status_string(int(status)).decode()
+    except ImportError:
+        return STATUS_NAMES.get(int(status), "PA_ERR_UNKNOWN")
+
+
+def pa_reshape_and_cache(key: torch.Tensor, value: torch.Tensor, slot_mapping: torch.Tensor,
+                         k_cache: torch.Tensor, v_cache: torch.Tensor, k_scale=None,
+                         v_scale=None, stream=None) -> None:
+    """key/value: [T, Hkv, D] (rows may be strided, e.g. views into a fused QKV
+    buffer); slot_mapping: int64 [T]; pools [NB, Hkv, 16, D]."""
+    assert key.stride() == value.stride() and key.stride(-1) == 1
+    T = key.shape[0]
+    desc = cache_desc(k_cache, k_scale, v_scale)
+    st = load_library().pa_reshape_and_cache(
+        _ptr(key), _ptr(value), dtype_code(key.dtype), T, key.stride(0) if T else 0,
+        _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache), ctypes.byref(desc), _stream(stream))
+    _check(st, "pa_reshape_and_cache")
+
+
+def pa_decode_workspace_size(batch: int, num_q_heads: int, head_dim: int, max_context_len: int,
+                             partition_size: int = 0) -> int:
+    return int(load_library().pa_decode_workspace_size(batch, num_q_heads, head_dim,
+                                                       max_context_len, partition_size))
+
+
+def pa_varlen_workspace_size(num_seqs: int, total_q: int, num_q_heads: int, head_dim: int,
+                             max_context_len: int) -> int:
+    return int(load_library().pa_varlen_workspace_size(num_seqs, total_q, num_q_heads, head_dim,
+                                                       max_context_len))
+
+
+def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]):
+    if nbytes == 0:
+        return workspace, 0 if workspace is None else workspace.numel()
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def pa_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+              block_tables: torch.Tensor, context_lens: torch.Tensor, max_context_len: int,
+              scale: float, k_scale=None, v_scale=None, partition_size: int = 0,
+              workspace: Optional[torch.Tensor] = None, stream=None) -> None:
+    """out/q: [B, Hq, D]; block_tables int32 [B, max_blocks]; context_lens int32 [B]."""
+    B, hq, d = q.shape
+    lib = load_library()
+    need = lib.pa_decode_workspace_size(B, hq, d, max_context_len, partition_size)
+    workspace, wbytes = _workspace(need, q.device, workspace)
+    desc = cache_desc(k_cache, k_scale, v_scale)
+    st = lib.pa_decode(_ptr(out), dtype_code(out.dtype), _ptr(q), dtype_code(q.dtype), B, hq,
+                       _ptr(k_cache), _ptr(v_cache), ctypes.byref(desc), _ptr(block_tables),
+                       block_tables.shape[1], _ptr(context_lens), int(max_context_len),
+                       float(scale), int(partition_size), _ptr(workspace), wbytes,
+                       _stream(stream))
+    _check(st, "pa_decode")
+
+
+def pa_varlen(out: torch.Tensor, q: torch.Tensor, cu_seqlens_q: torch.Tensor,
+              seqlens_k: torch.Tensor, max_q_len: int, max_context_len: int,
+              k_cache: torch.Tensor, v_cache: torch.Tensor, block_tables: torch.Tensor,
+              scale: float, k_scale=None, v_scale=None, workspace: Optional[torch.Tensor] = None,
+              stream=None) -> None:
+    """out/q: [total_q, Hq, D]; cu_seqlens_q int32 [S+1]; seqlens_k int32 [S]."""
+    total_q, hq, d = q.shape
+    S = seqlens_k.shape[0]
+    lib = load_library()
+    need = lib.pa_varlen_workspace_size(S, total_q, hq, d, max_context_len)
+    workspace, wbytes = _workspace(need, q.device, workspace)
+    desc = cache_desc(k_cache, k_scale, v_scale)
+    st = lib.pa_varlen(_ptr(out), dtype_code(out.dtype), _ptr(q), dtype_code(q.dtype), total_q,
+                       S, hq, _ptr(cu_seqlens_q), _ptr(seqlens_k), int(max_q_len),
+                       int(max_context_len), _ptr(k_cache), _ptr(v_cache), ctypes.byref(desc),
+                       _ptr(block_tables), block_tables.shape[1], float(scale), _ptr(workspace),
+                       wbytes, _stream(stream))
+    _check(st, "pa_varlen")
+
+
+def pa_device_error(stream=None) -> int:
+    """Read and clear the library's device error word (synchronises the stream)."""
+    return int(load_library().pa_device_error(_stream(stream)))

@@ -1,0 +1,122 @@
+"""The C-ABI library loads on a CPU-only host, exports every entry point its
+header declares, and answers the host-only calls (status strings, workspace
+sizing, argument validation) without touching a GPU."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from paged_kv_cache_lens_b200 import build as pa_build
+from paged_kv_cache_lens_b200 import pa
+
+
+@pytest.fixture(scope="module")
+def lib():
+    pa_build.build()
+    return pa.load_library()
+
+
+def test_header_declares_the_boundary():
+    names = pa.declared_functions()
+    for n in ["pa_reshape_and_cache", "pa_decode", "pa_varlen", "pa_decode_workspace_size",
+              "pa_varlen_workspace_size", "pa_status_string", "pa_device_error"]:
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in pa.declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_header_is_plain_c():
+    text = open(pa.HEADER).read()
+    assert 'extern "C"' in text
+    for bad in ("torch", "at::", "Tensor", "cuda_runtime", "cudaStream_t"):
+        assert bad not in re.sub(r"/\*.*?\*/", "", text, flags=re.S), bad
+
+
+def test_status_strings(lib):
+    for code, name in pa.STATUS_NAMES.items():
+        assert pa.pa_status_string(code).startswith(name)
+    assert pa.pa_status_string(99) == "PA_ERR_UNKNOWN"
+
+
+def test_decode_workspace_size_closed_form(lib):
+    # one partition (no split) needs no workspace
+    assert pa.pa_decode_workspace_size(64, 40, 128, 512, 512) == 0
+    # B*Hq*P floats for m and for l, B*Hq*P*D for o, each 256-aligned
+    B, H, D, L, P = 64, 40, 128, 2048, 512
+    parts = -(-L // P)
+    n = B * H * parts
+
+    def al(x):
+        return -(-x // 256) * 256
+    assert pa.pa_decode_workspace_size(B, H, D, L, P) == 2 * al(4 * n) + al(4 * n * D)
+    assert pa.pa_decode_workspace_size(B, H, D, L, 100) == 0     # invalid partition size
+    assert pa.pa_decode_workspace_size(0, H, D, L, P) == 0
+
+
+def test_varlen_workspace_size_includes_row_maps(lib):
+    got = pa.pa_varlen_workspace_size(204, 2248, 32, 128, 3584)
+    assert got >= 2 * 2248 * 4
+
+
+def _desc(**kw):
+    d = dict(num_blocks=64, block_size=16, num_kv_heads=2, head_dim=64, kv_dtype=pa.PA_F16,
+             k_scale=None, v_scale=None)
+    d.update(kw)
+    return pa.pa_cache_desc(**d)
+
+
+def test_host_validation_rejects_before_any_launch(lib):
+    P = ctypes.c_void_p
+    fake = P(0x10000)       # never dereferenced: every call below fails validation first
+    desc = _desc()
+    # null output
+    assert lib.pa_decode(None, 0, fake, 0, 4, 2, fake, fake, ctypes.byref(desc), fake, 8, fake,
+                         100, 0.125, 0, None, 0, None) == 1
+    # block size other than 16
+    bad = _desc(block_size=32)
+    assert lib.pa_decode(fake, 0, fake, 0, 4, 2, fake, fake, ctypes.byref(bad), fake, 8, fake,
+                         100, 0.125, 0, None, 0, None) == 2
+    # table too narrow for max_context_len
+    assert lib.pa_decode(fake, 0, fake, 0, 4, 2, fake, fake, ctypes.byref(desc), fake, 6, fake,
+                         100, 0.125, 0, None, 0, None) == 1
+    # q heads not a multiple of kv heads
+    assert lib.pa_decode(fake, 0, fake, 0, 4, 3, fake, fake, ctypes.byref(desc), fake, 8, fake,
+                         100, 0.125, 0, None, 0, None) == 1
+    # group of 16 heads is not built
+    assert lib.pa_decode(fake, 0, fake, 0, 4, 32, fake, fake, ctypes.byref(desc), fake, 8, fake,
+                         100, 0.125, 0, None, 0, None) == 2
+    # q dtype differs from a 16-bit pool
+    assert lib.pa_decode(fake, 0, fake, 1, 4, 2, fake, fake, ctypes.byref(desc), fake, 8, fake,
+                         100, 0.125, 0, None, 0, None) == 2
+    # bad partition size
+    assert lib.pa_decode(fake, 0, fake, 0, 4, 2, fake, fake, ctypes.byref(desc), fake, 8, fake,
+                         100, 0.125, 96, None, 0, None) == 1
+    # workspace needed (4 parts of 64) but missing
+    assert lib.pa_decode(fake, 0, fake, 0, 4, 2, fake, fake, ctypes.byref(desc), fake, 8, fake,
+                         100, 0.125, 64, None, 0, None) == 3
+    # FP8 pool without scales
+    f8 = _desc(kv_dtype=pa.PA_FP8_E4M3, head_dim=128)
+    assert lib.pa_decode(fake, 1, fake, 1, 4, 2, fake, fake, ctypes.byref(f8), fake, 8, fake,
+                         100, 0.125, 0, None, 0, None) == 1
+    # misaligned pool
+    assert lib.pa_decode(fake, 0, fake, 0, 4, 2, P(0x10002), fake, ctypes.byref(desc), fake, 8,
+                         fake, 100, 0.125, 0, None, 0, None) == 1
+    # reshape: stride smaller than a row, unsupported dtype pair
+    assert lib.pa_reshape_and_cache(fake, fake, 0, 4, 8, fake, fake, fake, ctypes.byref(desc),
+                                    None) == 1
+    assert lib.pa_reshape_and_cache(fake, fake, 1, 4, 128, fake, fake, fake, ctypes.byref(desc),
+                                    None) == 2
+    # zero work is a no-op success
+    assert lib.pa_reshape_and_cache(fake, fake, 0, 0, 128, fake, fake, fake, ctypes.byref(desc),
+                                    None) == 0
+    assert lib.pa_decode(fake, 0, fake, 0, 0, 2, fake, fake, ctypes.byref(desc), fake, 8, fake,
+                         100, 0.125, 0, None, 0, None) == 0
+    # varlen: workspace missing, q longer than context
+    assert lib.pa_varlen(fake, 0, fake, 0, 10, 2, 2, fake, fake, 5, 100, fake, fake,
+                         ctypes.byref(desc), fake, 8, 0.125, None, 0, None) == 3
+    assert lib.pa_varlen(fake, 0, fake, 0, 10, 2, 2, fake, fake, 200, 100, fake, fake,
+                         ctypes.byref(desc), fake, 8, 0.125, None, 0, None) == 1

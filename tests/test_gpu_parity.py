@@ -1,0 +1,280 @@
+"""GPU-vs-oracle parity of the hot path, called through the C ABI.
+
+Cache writes and indexing must match the oracle bit for bit; attention must
+be within max-abs 2e-3 (fp16/bf16 pools) or 5e-2 (FP8 pools) of the fp64
+oracle with fp32 output, plus half an output ulp when the output is 16-bit.
+"""
+import numpy as np
+import pytest
+import torch
+
+from paged_kv_cache_lens_b200 import pa
+from paged_kv_cache_lens_b200 import workloads as wl
+from tests._gpu import DeviceStep, assert_close, sampled_oracle_pools
+from tests._helpers import oracle_attention, oracle_pools
+
+pytestmark = pytest.mark.gpu
+
+F32 = wl.F32
+
+
+def _pool_bits(t):
+    return t.view(torch.uint8).cpu().numpy() if t.dtype == torch.uint8 else \
+        t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def _run_small(oracle, W, out_dtype=F32, partition_size=None):
+    d = DeviceStep(W, out_dtype=out_dtype)
+    d.fill_cache()
+    d.step(partition_size=partition_size)
+    torch.cuda.synchronize()
+    assert pa.pa_device_error() == 0
+    kc, vc = oracle_pools(oracle, W)
+    assert np.array_equal(_pool_bits(d.k_cache), kc), "K pool differs from the oracle's"
+    assert np.array_equal(_pool_bits(d.v_cache), vc), "V pool differs from the oracle's"
+    want = oracle_attention(oracle, W, kc, vc)
+    got = d.out_f64()
+    return assert_close(got, want, W, out_dtype, W.name), d
+
+
+# ---------------------------------------------------------------- cache write
+
+@pytest.mark.parametrize("kv", [wl.BF16, wl.F16, wl.FP8_E4M3])
+def test_reshape_and_cache_bit_exact(oracle, kv):
+    W = wl.build_workload("rc", 101, [1, 1, 1, 7], [1, 30, 64, 100], 8, 4, 128,
+                          dtype=wl.F16 if kv == wl.F16 else wl.BF16, kv_dtype=kv)
+    W.new_slots[2] = -1                          # a padding token is skipped
+    d = DeviceStep(W)
+    d.fill_cache()
+    d.write_new()
+    torch.cuda.synchronize()
+    kc, vc = oracle_pools(oracle, W)
+    assert np.array_equal(_pool_bits(d.k_cache), kc)
+    assert np.array_equal(_pool_bits(d.v_cache), vc)
+
+
+def test_reshape_and_cache_from_fused_qkv_rows(oracle):
+    rng = np.random.default_rng(7)
+    T, hq, hkv, D, nb = 37, 8, 2, 64, 16
+    qkv = wl.randn_bits(rng, (T, (hq + 2 * hkv) * D), wl.BF16)
+    slots = rng.choice(nb * 16, T, replace=False).astype(np.int64)
+    dev = torch.from_numpy(qkv.view(np.int16)).cuda().view(torch.bfloat16)
+    k = dev[:, hq * D:(hq + hkv) * D].view(T, hkv, D)
+    v = dev[:, (hq + hkv) * D:].view(T, hkv, D)
+    kc = torch.zeros((nb, hkv, 16, D), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    pa.pa_reshape_and_cache(k, v, torch.from_numpy(slots).cuda(), kc, vc)
+    ok_, ov_ = np.zeros((nb, hkv, 16, D), np.uint16), np.zeros((nb, hkv, 16, D), np.uint16)
+    oracle.reshape_and_cache(qkv[:, hq * D:], qkv[:, (hq + hkv) * D:], wl.BF16, slots, ok_, ov_,
+                             16, wl.BF16, token_stride=(hq + 2 * hkv) * D)
+    assert np.array_equal(_pool_bits(kc), ok_) and np.array_equal(_pool_bits(vc), ov_)
+
+
+# ---------------------------------------------------------------- decode
+
+def test_config1_tiny_mha_all_outputs(oracle):
+    W = wl.config(1)
+    for out_dtype in (F32, wl.F16):
+        _run_small(oracle, W, out_dtype)
+
+
+EDGE_LENS = [1, 15, 16, 17, 31, 32, 33, 63, 64, 65, 511, 512, 513, 1000]
+
+
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (8, 2), (16, 2), (6, 2)])
+@pytest.mark.parametrize("D", [64, 128, 256])
+def test_decode_edge_lengths(oracle, hq, hkv, D):
+    W = wl.build_workload("edge", 200 + D + hq, np.ones(len(EDGE_LENS), np.int64), EDGE_LENS, hq,
+                          hkv, D, dtype=wl.BF16)
+    for ps in (0, 64, 512):
+        _run_small(oracle, W, F32, partition_size=ps)
+
+
+@pytest.mark.parametrize("D", [128, 256])
+@pytest.mark.parametrize("q_dtype", [wl.BF16, wl.F16])
+def test_decode_fp8_pool(oracle, D, q_dtype):
+    W = wl.build_workload("fp8", 300 + D, np.ones(6, np.int64), [1, 17, 100, 513, 1024, 2000], 8,
+                          2, D, dtype=q_dtype, kv_dtype=wl.FP8_E4M3, out_dtype=wl.BF16)
+    for out_dtype in (F32, wl.BF16):
+        _run_small(oracle, W, out_dtype)
+
+
+def test_decode_f16(oracle):
+    W = wl.build_workload("f16", 77, np.ones(5, np.int64), [3, 40, 300, 700, 1500], 32, 8, 128,
+                          dtype=wl.F16)
+    _run_small(oracle, W, F32)
+    _run_small(oracle, W, wl.F16)
+
+
+def test_single_key_returns_value_exactly():
+    W = wl.build_workload("one", 5, np.ones(3, np.int64), [1, 1, 1], 8, 2, 128)
+    d = DeviceStep(W, out_dtype=wl.BF16)
+    d.fill_cache()
+    d.step()
+    torch.cuda.synchronize()
+    got = d.out.view(torch.int16).cpu().numpy().view(np.uint16)     # [3, 8, 128]
+    want = np.repeat(W.new_v, 4, axis=1)                              # KV head per group
+    assert np.array_equal(got, want)
+
+
+def test_zero_context_gives_zeros(oracle):
+    W = wl.build_workload("z", 6, np.ones(3, np.int64), [5, 40, 9], 4, 2, 64)
+    W.seqlens_k[1] = 0
+    _, d = _run_small(oracle, W, F32)
+    assert torch.all(d.out[1] == 0)
+
+
+def test_shared_prefix_equals_unshared_copies():
+    W = wl.build_workload("sp", 8, np.ones(4, np.int64), [300, 700, 513, 2048], 8, 2, 128,
+                          shared_prefix_len=256)
+    d = DeviceStep(W, out_dtype=F32)
+    d.fill_cache()
+    d.step()
+    shared = d.out.clone()
+    # copy the shared prefix blocks of requests 1..3 into fresh blocks
+    nb = W.num_blocks
+    extra = 3 * 16
+    kc = torch.cat([d.k_cache, torch.zeros((extra,) + d.k_cache.shape[1:], dtype=d.k_cache.dtype,
+                                           device="cuda")])
+    vc = torch.cat([d.v_cache, torch.zeros_like(kc[:extra])])
+    bt = W.block_tables.copy()
+    for j, r in enumerate([1, 2, 3]):
+        for i in range(16):
+            kc[nb + 16 * j + i] = kc[bt[r, i]]
+            vc[nb + 16 * j + i] = vc[bt[r, i]]
+            bt[r, i] = nb + 16 * j + i
+    out2 = torch.empty_like(d.out)
+    pa.pa_decode(out2, d.q, kc, vc, torch.from_numpy(bt).cuda(), d.seqlens_k, W.max_context_len,
+                 W.scale, workspace=d.workspace)
+    torch.cuda.synchronize()
+    assert torch.equal(shared, out2)
+
+
+def test_decode_is_deterministic(oracle):
+    W = wl.config(3, batch=16)
+    d = DeviceStep(W, out_dtype=F32)
+    d.fill_cache()
+    d.step()
+    a = d.out.clone()
+    d.attend()
+    torch.cuda.synchronize()
+    assert torch.equal(a, d.out)
+
+
+# ---------------------------------------------------------------- varlen
+
+def test_varlen_small_mixed(oracle):
+    q_lens = [1, 5, 17, 1, 33, 3, 64, 1, 100]
+    kv_lens = [1, 5, 50, 16, 33, 70, 64, 900, 611]     # chunk starts not multiples of 16
+    for hq, hkv, D in [(8, 2, 128), (4, 4, 64), (16, 2, 128)]:
+        W = wl.build_workload("vl", 400 + hq, q_lens, kv_lens, hq, hkv, D)
+        _run_small(oracle, W, F32)
+        _run_small(oracle, W, wl.BF16)
+
+
+def test_varlen_fp8(oracle):
+    W = wl.build_workload("vl8", 410, [1, 40, 1, 77], [600, 40, 33, 1100], 8, 2, 128,
+                          kv_dtype=wl.FP8_E4M3)
+    _run_small(oracle, W, F32)
+
+
+def test_varlen_decode_rows_equal_pa_decode():
+    """A varlen batch of q_len-1 requests reproduces pa_decode exactly."""
+    W = wl.config(3, batch=12)
+    d = DeviceStep(W, out_dtype=F32)
+    d.fill_cache()
+    d.step()
+    dec = d.out.clone()
+    out = torch.empty_like(dec)
+    pa.pa_varlen(out, d.q, d.cu, d.seqlens_k, 1, W.max_context_len, d.k_cache, d.v_cache,
+                 d.block_tables, W.scale)
+    torch.cuda.synchronize()
+    torch.testing.assert_close(out, dec, rtol=0, atol=2e-5)
+
+
+# ---------------------------------------------------------------- full sizes
+
+def _sample_rows(W, n, rng):
+    L = W.seqlens_k
+    picks = {int(np.argmax(L)), int(np.argmin(L))}
+    picks.update(int(x) for x in rng.choice(W.num_seqs, min(n, W.num_seqs), replace=False))
+    return sorted(picks)
+
+
+@pytest.mark.parametrize("cfg", [2, 3, 5])
+def test_full_size_decode_sampled(oracle, cfg):
+    """The reference workload at full size in the benchmark's launch
+    configuration; every output finite, sampled (row, head) pairs vs oracle."""
+    W = wl.config(cfg)
+    d = DeviceStep(W)
+    d.fill_cache()
+    d.step()
+    torch.cuda.synchronize()
+    assert pa.pa_device_error() == 0
+    got = d.out_f64()
+    assert np.isfinite(got).all()
+    rng = np.random.default_rng(cfg)
+    rows = _sample_rows(W, 6, rng)
+    kc, vc = sampled_oracle_pools(oracle, W, rows)
+    pr = np.repeat(rows, W.num_q_heads)
+    ph = np.tile(np.arange(W.num_q_heads), len(rows))
+    want = oracle_attention(oracle, W, kc, vc, pairs=(pr, ph), num_threads=8)
+    assert_close(got[pr, ph], want, W, W.out_dtype, W.name)
+
+
+def test_full_size_mixed_step_sampled(oracle):
+    W = wl.config(4)
+    d = DeviceStep(W)
+    d.fill_cache()
+    d.step()
+    torch.cuda.synchronize()
+    assert pa.pa_device_error() == 0
+    got = d.out_f64()
+    assert np.isfinite(got).all()
+    rng = np.random.default_rng(4)
+    dec_rows = sorted(rng.choice(200, 5, replace=False).tolist())
+    chunk_rows = []
+    for r in range(200, 204):
+        base = int(W.cu_seqlens_q[r])
+        chunk_rows += [base + i for i in (0, 1, 15, 16, 17, 255, 510, 511)]
+    rows = dec_rows + chunk_rows
+    kc, vc = sampled_oracle_pools(oracle, W, rows)
+    heads = [0, 3, 4, 17, 31]
+    pr = np.repeat(rows, len(heads))
+    ph = np.tile(heads, len(rows))
+    want = oracle_attention(oracle, W, kc, vc, pairs=(pr, ph), num_threads=8)
+    assert_close(got[pr, ph], want, W, W.out_dtype, W.name)
+
+
+# ---------------------------------------------------------------- errors
+
+def test_out_of_range_block_is_skipped_and_reported():
+    W = wl.build_workload("oob", 9, np.ones(2, np.int64), [40, 40], 4, 2, 64)
+    d = DeviceStep(W, out_dtype=F32)
+    d.fill_cache()
+    d.write_new()
+    bt = d.block_tables.clone()
+    bt[1, 1] = W.num_blocks + 5
+    pa.pa_decode(d.out, d.q, d.k_cache, d.v_cache, bt, d.seqlens_k, W.max_context_len, W.scale,
+                 workspace=d.workspace)
+    assert pa.pa_device_error() == 4
+    assert pa.pa_device_error() == 0                       # cleared by the read
+    assert torch.isfinite(d.out).all()
+
+
+def test_out_of_range_slot_is_skipped_and_reported():
+    W = wl.build_workload("oobs", 10, [1], [5], 2, 2, 64)
+    d = DeviceStep(W)
+    bad = torch.tensor([W.num_blocks * 16 + 3], dtype=torch.int64, device="cuda")
+    pa.pa_reshape_and_cache(d.new_k, d.new_v, bad, d.k_cache, d.v_cache)
+    assert pa.pa_device_error() == 4
+
+
+def test_workspace_too_small_is_rejected():
+    W = wl.build_workload("ws", 11, np.ones(2, np.int64), [2000, 3000], 8, 2, 128)
+    d = DeviceStep(W)
+    small = torch.empty(256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(pa.PaError) as e:
+        pa.pa_decode(d.out, d.q, d.k_cache, d.v_cache, d.block_tables, d.seqlens_k,
+                     W.max_context_len, W.scale, partition_size=512, workspace=small)
+    assert e.value.status == 3
