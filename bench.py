@@ -17,11 +17,13 @@ and reduced as the max over ranks.
 from __future__ import annotations
 
 import argparse
+import datetime
 import json
 import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -41,7 +43,7 @@ CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.ac
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", type=int, default=2, choices=[2, 3, 4, 5])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
@@ -78,27 +80,39 @@ def workload_name(W) -> str:
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+    """nvidia-smi samples of SM clock and throttle reasons.  Sampling starts
+    before the timed region; summary() keeps the samples stamped inside it
+    (widened by the sampling period, so a short region still gets one)."""
+
+    PERIOD_MS = 50
 
     def __init__(self, device_index: int):
         self.idx = device_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{device_index}.csv")
+        fd, self.path = tempfile.mkstemp(prefix=f"pa_clocks_{device_index}_", suffix=".csv")
+        os.close(fd)
+        self.t0 = self.t1 = None
 
-    def __enter__(self):
+    def start(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={CLOCK_QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu=timestamp,{CLOCK_QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", str(self.PERIOD_MS)],
                 stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.5)
         except OSError:
             self.proc = None
-        return self
 
-    def __exit__(self, *exc):
+    def mark_start(self):
+        self.t0 = datetime.datetime.now()
+
+    def mark_end(self):
+        self.t1 = datetime.datetime.now()
+
+    def stop(self):
         if self.proc is not None:
+            time.sleep(2 * self.PERIOD_MS / 1000)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -109,12 +123,20 @@ class ClockSampler:
     def summary(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        pad = datetime.timedelta(milliseconds=2 * self.PERIOD_MS)
         rows = []
         with open(self.path) as f:
             for line in f:
                 parts = [p.strip() for p in line.split(",")]
-                if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
-                    rows.append(parts)
+                if len(parts) < 10:
+                    continue
+                try:
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f")
+                    float(parts[2])
+                except ValueError:
+                    continue
+                if self.t0 - pad <= ts <= self.t1 + pad:
+                    rows.append(parts[1:])
         if not rows:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
         sm = [float(r[1]) for r in rows]
@@ -228,26 +250,28 @@ def run_native(args):
     max_parts = -(-W.max_context_len // (W.partition_size or 512))
     launches_per_step = 1 + 1 + (1 if max_parts > 1 else 0) + (0 if W.decode else 1)
 
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize(dev)
-
     # ---- device-timed region: K whole steps, attention launches timed too
     ev_a = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
             for _ in range(args.steps)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(local) as clocks:
-        barrier(world)
-        torch.cuda.synchronize(dev)
-        t0.record(stream)
-        for i in range(args.steps):
-            pa.pa_reshape_and_cache(nk, nv, slots, kc, vc, ks, vs, stream)
-            ev_a[i][0].record(stream)
-            attend(q, bt, sk, cu, out)
-            ev_a[i][1].record(stream)
-        t1.record(stream)
-        torch.cuda.synchronize(dev)
-        barrier(world)
+    clocks = ClockSampler(local)
+    clocks.start()
+    for _ in range(args.warmup):
+        step()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    clocks.mark_start()
+    t0.record(stream)
+    for i in range(args.steps):
+        pa.pa_reshape_and_cache(nk, nv, slots, kc, vc, ks, vs, stream)
+        ev_a[i][0].record(stream)
+        attend(q, bt, sk, cu, out)
+        ev_a[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.mark_end()
+    barrier(world)
+    clocks.stop()
     ms_local = t0.elapsed_time(t1) / args.steps
     attn_ms = float(np.mean([a.elapsed_time(b) for a, b in ev_a]))
     ms = max_over_ranks(ms_local, world)
@@ -416,16 +440,23 @@ def _oracle_sample(W, n_seqs, threads):
 
 
 def cpu_baseline(W, budget_s=12.0):
+    """The oracle, as it stands, on this host's cores: a sample of the step
+    (first n requests) grown towards budget_s, then repeated until the budget
+    is spent."""
     threads = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
-    n = 1
-    t, b, reqs = _oracle_sample(W, n, threads)
-    # grow the sample to roughly the time budget (bounded by the batch)
-    if t < budget_s and n < W.num_seqs:
-        n = int(min(W.num_seqs, max(2, budget_s / max(t, 1e-3))))
+    t, b, reqs = _oracle_sample(W, 1, threads)
+    if t < budget_s and reqs < W.num_seqs:
+        n = int(min(W.num_seqs, max(2, 0.5 * budget_s / max(t, 1e-3))))
         t, b, reqs = _oracle_sample(W, n, threads)
-    return {"value": round(b / t / 1e9, 4), "unit": "GB/s", "cores": threads, "kind": "oracle",
+    total_t, total_b, reps = t, b, 1
+    while total_t < budget_s:
+        t, b, reqs = _oracle_sample(W, reqs, threads)
+        total_t, total_b, reps = total_t + t, total_b + b, reps + 1
+    return {"value": round(total_b / total_t / 1e9, 4), "unit": "GB/s", "cores": threads,
+            "kind": "oracle",
             "sample": f"{reqs} of {W.num_seqs} requests of the step (cache write + attention, "
-                      f"fp64), {t:.1f} s", "seq_steps_per_s_per_layer": round(reqs / t, 3)}
+                      f"fp64) x {reps} repeats, {total_t:.1f} s",
+            "seq_steps_per_s_per_layer": round(reqs * reps / total_t, 3)}
 
 
 def run_reference(args):
