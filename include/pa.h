@@ -187,6 +187,37 @@ pa_status pa_varlen(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dty
                     size_t workspace_bytes, void* stream);
 
 /*
+ * Size of the fixed device scratch behind pa_decode_static (per GPU).
+ */
+#define PA_DECODE_STATIC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+/*
+ * pa_decode without a workspace argument, for callers that cannot allocate
+ * device memory (the pages describe no such call; it exists for this
+ * library's users).  A plug-in inside a host program that owns all device
+ * memory and exposes no allocator, or a latency-critical loop that cannot
+ * afford cudaMalloc's implicit device synchronisation, still has to hand
+ * pa_decode a workspace; this call instead keeps its split-K partials in a
+ * file-scope device array of PA_DECODE_STATIC_SCRATCH_BYTES that every GPU
+ * loading the library holds until the process exits.  It allocates nothing.
+ *
+ * Arguments and results are those of pa_decode minus the workspace.  Sizes
+ * whose partials need more than PA_DECODE_STATIC_SCRATCH_BYTES (see
+ * pa_decode_workspace_size) return PA_ERR_WORKSPACE without launching.
+ * The first call on each device, made with that device current, looks up
+ * the array's device address (cudaGetSymbolAddress); make that first call
+ * before any stream capture.  All calls on one device share the array and
+ * leave their partials in it: calls that overlap on the GPU (other streams,
+ * other host threads) race and must be serialised by the caller.
+ */
+pa_status pa_decode_static(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dtype,
+                           int32_t batch, int32_t num_q_heads, const void* k_cache,
+                           const void* v_cache, const pa_cache_desc* cache,
+                           const int32_t* block_tables, int32_t max_blocks_per_seq,
+                           const int32_t* context_lens, int32_t max_context_len, float scale,
+                           int32_t partition_size, void* stream);
+
+/*
  * Read and clear the device error word that kernels set when they skip an
  * out-of-range block id or slot (PA_ERR_OUT_OF_RANGE) or give up a bounded
  * wait (PA_ERR_TIMEOUT).  Synchronises `stream` first.  Returns PA_OK when no
