@@ -47,6 +47,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", type=int, default=2, choices=[2, 3, 4, 5])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--batch", type=int, default=None,
+                    help="fewer requests, same distributions (profiling captures only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -193,7 +195,7 @@ def run_native(args):
 
     rank, world, local = dist_setup(args.gpus)
     dev = torch.device("cuda", local if world > 1 else 0)
-    W = wl.config(args.workload)
+    W = wl.config(args.workload, batch=args.batch)
     TD = {wl.F16: torch.float16, wl.BF16: torch.bfloat16, wl.F32: torch.float32}
 
     def to_dev(a, dt):

@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 
 #include <climits>
+#include <cstdio>
+#include <cstdlib>
 #include <cstdint>
 #include <cstring>
 
@@ -55,6 +57,19 @@ EncodeTiledFn encode_fn() {
       fn = reinterpret_cast<EncodeTiledFn>(p);
   }
   return fn;
+}
+
+// With PA_DEBUG set in the environment, CUDA failures are described on stderr
+// (the status code alone cannot carry the runtime's reason).
+pa_status cuda_fail(cudaError_t e, const char* where) {
+  if (std::getenv("PA_DEBUG"))
+    std::fprintf(stderr, "libpa: %s: %s\n", where, cudaGetErrorString(e));
+  return PA_ERR_CUDA;
+}
+
+pa_status map_fail(const char* which) {
+  if (std::getenv("PA_DEBUG")) std::fprintf(stderr, "libpa: tensor map for %s failed\n", which);
+  return PA_ERR_CUDA;
 }
 
 size_t elem_size(pa_dtype t) {
@@ -106,6 +121,26 @@ bool make_pool_tensor_map(CUtensorMap* map, const void* base, int kv_dtype, int6
                    2, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS && std::getenv("PA_DEBUG"))
+    std::fprintf(stderr, "libpa: pool tensor map: CUresult %d\n", static_cast<int>(r));
+  return r == CUDA_SUCCESS;
+}
+
+bool make_q_tensor_map(CUtensorMap* map, const void* q, int64_t total_q, int32_t num_q_heads,
+                       int32_t head_dim, int32_t group, int32_t rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(num_q_heads),
+                        static_cast<cuuint64_t>(total_q)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2,
+                           static_cast<cuuint64_t>(num_q_heads) * head_dim * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(group), static_cast<cuuint32_t>(rows)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(q), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS && std::getenv("PA_DEBUG"))
+    std::fprintf(stderr, "libpa: q tensor map: CUresult %d\n", static_cast<int>(r));
   return r == CUDA_SUCCESS;
 }
 
@@ -151,7 +186,7 @@ pa_status pa_reshape_and_cache(const void* key, const void* value, pa_dtype src_
       key, value, src_dtype, num_tokens, token_stride, slot_mapping, k_cache, v_cache,
       cache->num_blocks, cache->block_size, cache->num_kv_heads, cache->head_dim,
       cache->kv_dtype, cache->k_scale, cache->v_scale, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return e == cudaSuccess ? PA_OK : cuda_fail(e, "reshape_and_cache launch");
 }
 
 size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t head_dim,
@@ -219,9 +254,9 @@ static pa_status run_attention(AttnArgs& a, const pa_cache_desc* cache, int32_t 
                             kBlockSize) ||
       !make_pool_tensor_map(&vmap, a.v_cache, cache->kv_dtype, pool_rows, cache->head_dim,
                             kBlockSize))
-    return PA_ERR_CUDA;
+    return map_fail("the KV pool");
   cudaError_t e = launch_paged_attention(a, kmap, vmap, stream);
-  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
+  return e == cudaSuccess ? PA_OK : cuda_fail(e, "attention launch");
 }
 
 static void fill_common(AttnArgs& a, void* out, pa_dtype out_dtype, const void* q,
@@ -300,9 +335,12 @@ pa_status pa_varlen(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dty
   int32_t* row_seq = reinterpret_cast<int32_t*>(b);
   int32_t* row_len = reinterpret_cast<int32_t*>(b + map_bytes);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (launch_varlen_prep(total_q, num_seqs, cu_seqlens_q, seqlens_k, row_seq, row_len, s) !=
-      cudaSuccess)
-    return PA_ERR_CUDA;
+  const int32_t group = num_q_heads / cache->num_kv_heads;
+  const bool chunks = max_q_len >= 2 && aligned(out, 16) &&
+                      prefill_supported(q_dtype, cache->kv_dtype, cache->head_dim, group);
+  cudaError_t pe = launch_varlen_prep(total_q, num_seqs, cu_seqlens_q, seqlens_k, row_seq,
+                                      row_len, chunks, s);
+  if (pe != cudaSuccess) return cuda_fail(pe, "varlen row map launch");
   AttnArgs a;
   fill_common(a, out, out_dtype, q, q_dtype, num_q_heads, k_cache, v_cache, cache, block_tables,
               max_blocks_per_seq, scale);
@@ -312,6 +350,23 @@ pa_status pa_varlen(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dty
   a.row_len = row_len;
   a.cu_seqlens_q = cu_seqlens_q;
   a.seqlens_k = seqlens_k;
+  if (chunks) {
+    // q_len >= 2 requests: one tensor-core kernel over (request, head, query tile)
+    const int64_t pool_rows =
+        static_cast<int64_t>(cache->num_blocks) * cache->num_kv_heads * kBlockSize;
+    CUtensorMap kmap, vmap, qmap;
+    if (!make_pool_tensor_map(&kmap, k_cache, cache->kv_dtype, pool_rows, cache->head_dim,
+                              kBlockSize) ||
+        !make_pool_tensor_map(&vmap, v_cache, cache->kv_dtype, pool_rows, cache->head_dim,
+                              kBlockSize) ||
+        !make_q_tensor_map(&qmap, q, total_q, num_q_heads, cache->head_dim, group,
+                           prefill_query_tile(group)))
+      return map_fail("the prefill operands");
+    AttnArgs p = a;
+    p.max_context_len = max_context_len;
+    cudaError_t fe = launch_paged_prefill(p, kmap, vmap, qmap, max_q_len, s);
+    if (fe != cudaSuccess) return cuda_fail(fe, "prefill launch");
+  }
   const int32_t ps = auto_partition(total_q, num_q_heads, max_context_len);
   return run_attention(a, cache, max_context_len, ps,
                        reinterpret_cast<float*>(b + 2 * map_bytes),

@@ -56,9 +56,22 @@ bool make_pool_tensor_map(CUtensorMap* map, const void* base, int kv_dtype, int6
 cudaError_t launch_paged_attention(const AttnArgs& a, const CUtensorMap& kmap,
                                    const CUtensorMap& vmap, cudaStream_t stream);
 
+// Request and visible-key count of each packed row.  With skip_chunks, rows
+// of requests with q_len >= 2 get row_len = -1 (the prefill kernel owns them).
 cudaError_t launch_varlen_prep(int32_t total_q, int32_t num_seqs, const int32_t* cu_seqlens_q,
                                const int32_t* seqlens_k, int32_t* row_seq, int32_t* row_len,
-                               cudaStream_t stream);
+                               bool skip_chunks, cudaStream_t stream);
+
+// Tensor-core prefill of the q_len >= 2 requests of a varlen step.
+bool prefill_supported(int q_dtype, int kv_dtype, int32_t head_dim, int32_t group);
+int prefill_query_tile(int32_t group);
+cudaError_t launch_paged_prefill(const AttnArgs& a, const CUtensorMap& kmap,
+                                 const CUtensorMap& vmap, const CUtensorMap& qmap,
+                                 int32_t max_q_len, cudaStream_t stream);
+
+// 3-D tensor map over q [total_q][Hq][D] (16-bit), box {64, group, rows}.
+bool make_q_tensor_map(CUtensorMap* map, const void* q, int64_t total_q, int32_t num_q_heads,
+                       int32_t head_dim, int32_t group, int32_t rows);
 
 cudaError_t launch_reshape_and_cache(const void* key, const void* value, int src_dtype,
                                      int64_t num_tokens, int64_t token_stride,

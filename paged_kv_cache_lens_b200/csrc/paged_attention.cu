@@ -111,6 +111,7 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
     seq = row;
     L = a.context_lens[row];
   }
+  if (L < 0) return;               // a varlen row owned by the prefill kernel
   L = min(L, a.max_context_len);   // a row longer than the promised bound is cut there
   const int group = a.group;
   const int hq0 = h * group;
@@ -535,7 +536,7 @@ __global__ void __launch_bounds__(kThreads) lse_reduce_kernel(const __grid_const
 // Request index and visible-key count of every packed query row.
 __global__ void varlen_prep_kernel(int32_t total_q, int32_t num_seqs, const int32_t* cu,
                                    const int32_t* seqlens_k, int32_t* row_seq,
-                                   int32_t* row_len) {
+                                   int32_t* row_len, bool skip_chunks) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= total_q) return;
   int lo = 0, hi = num_seqs;            // first r with cu[r] > i, minus one
@@ -551,7 +552,7 @@ __global__ void varlen_prep_kernel(int32_t total_q, int32_t num_seqs, const int3
   int n = kv - q_len + (i - cu[r]) + 1;
   n = n < 0 ? 0 : (n > kv ? kv : n);
   row_seq[i] = r;
-  row_len[i] = n;
+  row_len[i] = (skip_chunks && q_len >= 2) ? -1 : n;
 }
 
 template <int KVT, bool Q_BF16, int D, int GT>
@@ -630,11 +631,11 @@ cudaError_t launch_paged_attention(const AttnArgs& a, const CUtensorMap& kmap,
 
 cudaError_t launch_varlen_prep(int32_t total_q, int32_t num_seqs, const int32_t* cu_seqlens_q,
                                const int32_t* seqlens_k, int32_t* row_seq, int32_t* row_len,
-                               cudaStream_t stream) {
+                               bool skip_chunks, cudaStream_t stream) {
   if (total_q <= 0) return cudaSuccess;
   const int threads = 256;
   varlen_prep_kernel<<<(total_q + threads - 1) / threads, threads, 0, stream>>>(
-      total_q, num_seqs, cu_seqlens_q, seqlens_k, row_seq, row_len);
+      total_q, num_seqs, cu_seqlens_q, seqlens_k, row_seq, row_len, skip_chunks);
   return cudaGetLastError();
 }
 

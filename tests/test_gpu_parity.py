@@ -166,10 +166,20 @@ def test_decode_is_deterministic(oracle):
 def test_varlen_small_mixed(oracle):
     q_lens = [1, 5, 17, 1, 33, 3, 64, 1, 100]
     kv_lens = [1, 5, 50, 16, 33, 70, 64, 900, 611]     # chunk starts not multiples of 16
-    for hq, hkv, D in [(8, 2, 128), (4, 4, 64), (16, 2, 128)]:
+    for hq, hkv, D in [(8, 2, 128), (4, 4, 64), (16, 2, 128), (8, 8, 128), (8, 4, 128)]:
         W = wl.build_workload("vl", 400 + hq, q_lens, kv_lens, hq, hkv, D)
         _run_small(oracle, W, F32)
         _run_small(oracle, W, wl.BF16)
+
+
+@pytest.mark.parametrize("hq,hkv", [(4, 4), (8, 4), (32, 8), (16, 2)])
+def test_varlen_long_chunks(oracle, hq, hkv):
+    """Chunks longer than one query tile, over cached context that is not a
+    multiple of the block or key-tile size, with a decode row beside them."""
+    q_lens = [300, 1, 130, 257]
+    kv_lens = [300 + 77, 1000, 130 + 400, 257 + 129]
+    W = wl.build_workload("vlong", 420 + hq, q_lens, kv_lens, hq, hkv, 128)
+    _run_small(oracle, W, F32)
 
 
 def test_varlen_fp8(oracle):
