@@ -198,15 +198,26 @@ size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t head
   return decode_workspace_layout(batch, num_q_heads, head_dim, parts).total;
 }
 
+// Varlen workspace: [row_seq | row_len] int32 [total_q] each, the prefill
+// work list (int2 [capacity] + a count), then the split-K partials for
+// max(total_q, num_seqs) rows.
+static int64_t varlen_rows(int32_t num_seqs, int32_t total_q) {
+  return total_q > num_seqs ? total_q : num_seqs;
+}
+
 size_t pa_varlen_workspace_size(int32_t num_seqs, int32_t total_q, int32_t num_q_heads,
                                 int32_t head_dim, int32_t max_context_len) {
   if (num_seqs <= 0 || total_q <= 0 || num_q_heads <= 0 || head_dim <= 0) return 0;
   const int64_t maps = 2 * align_up(static_cast<int64_t>(total_q) * 4, kAlign);
-  if (max_context_len <= 0) return static_cast<size_t>(maps);
-  const int32_t ps = auto_partition(total_q, num_q_heads, max_context_len);
+  const int64_t items =
+      align_up(static_cast<int64_t>(prefill_item_capacity(num_seqs, total_q)) * 8, kAlign) +
+      kAlign;
+  if (max_context_len <= 0) return static_cast<size_t>(maps + items);
+  const int64_t rows = varlen_rows(num_seqs, total_q);
+  const int32_t ps = auto_partition(rows, num_q_heads, max_context_len);
   const int32_t parts = static_cast<int32_t>(cdiv(max_context_len, ps));
-  return static_cast<size_t>(maps) +
-         decode_workspace_layout(total_q, num_q_heads, head_dim, parts).total;
+  return static_cast<size_t>(maps + items) +
+         decode_workspace_layout(rows, num_q_heads, head_dim, parts).total;
 }
 
 static pa_status check_attention(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dtype,
@@ -332,26 +343,27 @@ pa_status pa_varlen(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dty
   if (!aligned(workspace, 256)) return PA_ERR_INVALID_ARG;
   auto* b = static_cast<uint8_t*>(workspace);
   const int64_t map_bytes = align_up(static_cast<int64_t>(total_q) * 4, kAlign);
+  const int32_t capacity = prefill_item_capacity(num_seqs, total_q);
+  const int64_t item_bytes = align_up(static_cast<int64_t>(capacity) * 8, kAlign) + kAlign;
   int32_t* row_seq = reinterpret_cast<int32_t*>(b);
   int32_t* row_len = reinterpret_cast<int32_t*>(b + map_bytes);
+  int2* items = reinterpret_cast<int2*>(b + 2 * map_bytes);
+  int32_t* item_count = reinterpret_cast<int32_t*>(b + 2 * map_bytes + item_bytes - kAlign);
+  uint8_t* partials = b + 2 * map_bytes + item_bytes;
+  const size_t head = static_cast<size_t>(2 * map_bytes + item_bytes);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int32_t group = num_q_heads / cache->num_kv_heads;
-  const bool chunks = max_q_len >= 2 && aligned(out, 16) &&
+  const bool chunks = max_q_len >= 2 && scale > 0.f && aligned(out, 16) &&
                       prefill_supported(q_dtype, cache->kv_dtype, cache->head_dim, group);
-  cudaError_t pe = launch_varlen_prep(total_q, num_seqs, cu_seqlens_q, seqlens_k, row_seq,
-                                      row_len, chunks, s);
-  if (pe != cudaSuccess) return cuda_fail(pe, "varlen row map launch");
   AttnArgs a;
   fill_common(a, out, out_dtype, q, q_dtype, num_q_heads, k_cache, v_cache, cache, block_tables,
               max_blocks_per_seq, scale);
-  a.rows = total_q;
   a.num_seqs = num_seqs;
-  a.row_seq = row_seq;
-  a.row_len = row_len;
   a.cu_seqlens_q = cu_seqlens_q;
   a.seqlens_k = seqlens_k;
   if (chunks) {
-    // q_len >= 2 requests: one tensor-core kernel over (request, head, query tile)
+    // q_len >= 2 requests: the tensor-core prefill over a compact work list;
+    // q_len == 1 requests: the decode kernel, one work row per request.
     const int64_t pool_rows =
         static_cast<int64_t>(cache->num_blocks) * cache->num_kv_heads * kBlockSize;
     CUtensorMap kmap, vmap, qmap;
@@ -364,13 +376,25 @@ pa_status pa_varlen(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dty
       return map_fail("the prefill operands");
     AttnArgs p = a;
     p.max_context_len = max_context_len;
-    cudaError_t fe = launch_paged_prefill(p, kmap, vmap, qmap, max_q_len, s);
+    p.pf_items = items;
+    p.pf_count = item_count;
+    cudaError_t fe = launch_paged_prefill(p, kmap, vmap, qmap, capacity, s);
     if (fe != cudaSuccess) return cuda_fail(fe, "prefill launch");
+    a.rows = num_seqs;
+    a.varlen_requests = 1;
+  } else {
+    cudaError_t pe = launch_varlen_prep(total_q, num_seqs, cu_seqlens_q, seqlens_k, row_seq,
+                                        row_len, false, s);
+    if (pe != cudaSuccess) return cuda_fail(pe, "varlen row map launch");
+    a.rows = total_q;
+    a.row_seq = row_seq;
+    a.row_len = row_len;
   }
-  const int32_t ps = auto_partition(total_q, num_q_heads, max_context_len);
-  return run_attention(a, cache, max_context_len, ps,
-                       reinterpret_cast<float*>(b + 2 * map_bytes),
-                       workspace_bytes - 2 * map_bytes, need - 2 * map_bytes, s);
+  const int32_t ps = auto_partition(varlen_rows(num_seqs, total_q), num_q_heads, max_context_len);
+  const int32_t parts = static_cast<int32_t>(cdiv(max_context_len > 0 ? max_context_len : 1, ps));
+  const size_t part_need = decode_workspace_layout(a.rows, num_q_heads, cache->head_dim, parts).total;
+  return run_attention(a, cache, max_context_len, ps, reinterpret_cast<float*>(partials),
+                       workspace_bytes - head, part_need, s);
 }
 
 pa_status pa_device_error(void* stream) {

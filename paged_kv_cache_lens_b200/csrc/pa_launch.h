@@ -26,6 +26,9 @@ struct AttnArgs {
   const int32_t* row_len;       // varlen: visible keys of each row (workspace)
   const int32_t* cu_seqlens_q;  // varlen only
   const int32_t* seqlens_k;     // varlen only
+  int32_t varlen_requests;      // varlen, chunk path on: row index = request, q_len 1 only
+  const int2* pf_items;         // prefill work list (request, query tile)
+  const int32_t* pf_count;      // number of valid items
   int32_t num_seqs;
   const float* k_scale;
   const float* v_scale;
@@ -65,9 +68,12 @@ cudaError_t launch_varlen_prep(int32_t total_q, int32_t num_seqs, const int32_t*
 // Tensor-core prefill of the q_len >= 2 requests of a varlen step.
 bool prefill_supported(int q_dtype, int kv_dtype, int32_t head_dim, int32_t group);
 int prefill_query_tile(int32_t group);
+int32_t prefill_item_capacity(int32_t num_seqs, int32_t total_q);
+// Builds the (request, query tile) list in a.pf_items / a.pf_count, then runs
+// the tensor-core prefill over it (grid = capacity x KV heads).
 cudaError_t launch_paged_prefill(const AttnArgs& a, const CUtensorMap& kmap,
                                  const CUtensorMap& vmap, const CUtensorMap& qmap,
-                                 int32_t max_q_len, cudaStream_t stream);
+                                 int32_t capacity, cudaStream_t stream);
 
 // 3-D tensor map over q [total_q][Hq][D] (16-bit), box {64, group, rows}.
 bool make_q_tensor_map(CUtensorMap* map, const void* q, int64_t total_q, int32_t num_q_heads,

@@ -71,6 +71,28 @@ __device__ __forceinline__ int swz(int row, int chunk) {  // 128-byte swizzle
   return row * 128 + ((chunk ^ (row & 7)) << 4);
 }
 
+// The sequence, visible-key count and packed query row behind work row `row`:
+// decode (row = sequence), varlen rows mapped by the row-map kernel, or varlen
+// requests with the chunk path on (row = request; only q_len-1 requests here,
+// L = -1 marks the others, which the prefill kernel owns).
+__device__ __forceinline__ void resolve_row(const AttnArgs& a, int row, int& seq, int& L,
+                                            int& qrow) {
+  if (a.row_seq) {
+    seq = a.row_seq[row];
+    L = a.row_len[row];
+    qrow = row;
+  } else if (a.varlen_requests) {
+    seq = row;
+    const int c0 = a.cu_seqlens_q[row];
+    qrow = c0;
+    L = (a.cu_seqlens_q[row + 1] - c0 == 1) ? a.seqlens_k[row] : -1;
+  } else {
+    seq = row;
+    L = a.context_lens[row];
+    qrow = row;
+  }
+}
+
 template <int KVT, bool Q_BF16, int D, int GT, int NSTAGE>
 __global__ void __launch_bounds__(kThreads)
 paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUtensorMap kmap,
@@ -103,14 +125,8 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
   bid /= a.max_parts;
   const int h = static_cast<int>(bid % a.num_kv_heads);
   const int row = static_cast<int>(bid / a.num_kv_heads);
-  int seq, L;
-  if (a.row_seq) {
-    seq = a.row_seq[row];
-    L = a.row_len[row];
-  } else {
-    seq = row;
-    L = a.context_lens[row];
-  }
+  int seq, L, qrow;
+  resolve_row(a, row, seq, L, qrow);
   if (L < 0) return;               // a varlen row owned by the prefill kernel
   L = min(L, a.max_context_len);   // a row longer than the promised bound is cut there
   const int group = a.group;
@@ -119,7 +135,7 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
   if (L <= 0) {
     if (part == 0)
       for (int i = threadIdx.x; i < group * D; i += kThreads)
-        store_out(a.out, (static_cast<int64_t>(row) * Hq + hq0) * D + i, a.out_dtype, 0.f);
+        store_out(a.out, (static_cast<int64_t>(qrow) * Hq + hq0) * D + i, a.out_dtype, 0.f);
     return;
   }
   const int PS = a.partition_size;
@@ -173,13 +189,13 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
   {
     const int n = r;
     const bool live = n < group && n < GT;
-    const uint16_t* qrow = static_cast<const uint16_t*>(a.q) +
-                           (static_cast<int64_t>(row) * Hq + hq0 + (live ? n : 0)) * D;
+    const uint16_t* qptr = static_cast<const uint16_t*>(a.q) +
+                           (static_cast<int64_t>(qrow) * Hq + hq0 + (live ? n : 0)) * D;
     if constexpr (!kFP8) {
 #pragma unroll
       for (int p = 0; p < D / 32; ++p) {
         const int base = (p >> 1) * 64 + 8 * (2 * c + (p & 1));
-        uint4 w = live ? *reinterpret_cast<const uint4*>(qrow + base) : make_uint4(0, 0, 0, 0);
+        uint4 w = live ? *reinterpret_cast<const uint4*>(qptr + base) : make_uint4(0, 0, 0, 0);
         qf[2 * p][0] = w.x;
         qf[2 * p][1] = w.y;
         qf[2 * p + 1][0] = w.z;
@@ -191,8 +207,8 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
         const int base = (p >> 1) * 128 + 16 * (2 * c + (p & 1));
         uint4 w0 = make_uint4(0, 0, 0, 0), w1 = w0;
         if (live) {
-          w0 = *reinterpret_cast<const uint4*>(qrow + base);
-          w1 = *reinterpret_cast<const uint4*>(qrow + base + 8);
+          w0 = *reinterpret_cast<const uint4*>(qptr + base);
+          w1 = *reinterpret_cast<const uint4*>(qptr + base + 8);
         }
         uint32_t wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
@@ -484,10 +500,11 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
       lsum += f * mg[w * stride_w + GT * D + GT + g];
       o += f * mg[w * stride_w + g * D + d];
     }
-    const int64_t hq = static_cast<int64_t>(row) * Hq + hq0 + g;
     if (single) {
-      store_out(a.out, hq * D + d, a.out_dtype, lsum > 0.f ? o * v_mul / lsum : 0.f);
+      const int64_t oq = static_cast<int64_t>(qrow) * Hq + hq0 + g;
+      store_out(a.out, oq * D + d, a.out_dtype, lsum > 0.f ? o * v_mul / lsum : 0.f);
     } else {
+      const int64_t hq = static_cast<int64_t>(row) * Hq + hq0 + g;
       const int64_t pidx = hq * a.max_parts + part;
       a.ws_o[pidx * D + d] = o;
       if (d == 0) {
@@ -503,7 +520,9 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
 __global__ void __launch_bounds__(kThreads) lse_reduce_kernel(const __grid_constant__ AttnArgs a) {
   const int h = blockIdx.x % a.num_kv_heads;
   const int row = blockIdx.x / a.num_kv_heads;
-  const int L = min(a.row_seq ? a.row_len[row] : a.context_lens[row], a.max_context_len);
+  int seq, L, qrow;
+  resolve_row(a, row, seq, L, qrow);
+  L = min(L, a.max_context_len);
   const int PS = a.partition_size;
   const int nparts = (L + PS - 1) / PS;
   if (nparts <= 1) return;
@@ -529,7 +548,8 @@ __global__ void __launch_bounds__(kThreads) lse_reduce_kernel(const __grid_const
     float o = 0.f;
     for (int p = 0; p < nparts; ++p)
       o += fast_exp2(a.ws_m[base + p] - s_M[g]) * a.ws_o[(base + p) * D + d];
-    store_out(a.out, hq * D + d, a.out_dtype, o * s_inv[g]);
+    const int64_t oq = static_cast<int64_t>(qrow) * Hq + hq0 + g;
+    store_out(a.out, oq * D + d, a.out_dtype, o * s_inv[g]);
   }
 }
 

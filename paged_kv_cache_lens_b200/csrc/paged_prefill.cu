@@ -29,21 +29,34 @@
 namespace pa {
 namespace {
 
-constexpr int kPfThreads = 192;          // 4 softmax warps, 1 TMA warp, 1 MMA warp
+constexpr int kSoftmaxWarps = 8;         // two warps per TMEM lane quarter, 64 columns each
+constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
+constexpr int kProducerWarps = 4;        // TMA issue is spread over 4 warps (2 blocks each)
+constexpr int kProducerWarp0 = 8;
+constexpr int kMmaWarp = kProducerWarp0 + kProducerWarps;
+constexpr int kPfThreads = (kMmaWarp + 1) * 32;
 constexpr int kBN = 128;                 // keys per tile
 constexpr int kHalf = 128 * 128;         // one 64-column (128-byte) half of a 128-row tile
 constexpr int kQBytes = 2 * kHalf;
-constexpr int kKVBytes = 2 * kHalf;
-constexpr int kStageBytes = 2 * kKVBytes;
-constexpr int kStages = 2;
-constexpr int kBarBase = kQBytes + kStages * kStageBytes;
-constexpr int kNumBars = 12;
+constexpr int kTileBytes = 2 * kHalf;    // one K or V tile: 128 keys x 128 dims
+constexpr int kKStages = 3;              // K is freed as soon as S is computed
+constexpr int kVStages = 2;              // V is freed when PV has run
+constexpr int kSBufs = 3;                // S/P buffers in TMEM
+constexpr int kKOff = kQBytes;
+constexpr int kVOff = kKOff + kKStages * kTileBytes;
+constexpr int kTblMax = 2048;            // block-table entries cached in shared memory
+constexpr int kTblOff = kVOff + kVStages * kTileBytes;
+constexpr int kRedOff = kTblOff + kTblMax * 4;          // [2][128] floats, max then sum
+constexpr int kBarBase = kRedOff + 2 * 128 * 4;
+// barriers: Q | K full x3 | K empty x3 | V full x2 | V empty x2 | S full x3 | P full x3 |
+//           PV done x3 | O
+enum { B_Q = 0, B_KF = 1, B_KE = 4, B_VF = 7, B_VE = 9, B_SF = 11, B_PF = 14, B_PVD = 17,
+       B_O = 20, kNumBars = 21 };
 constexpr int kSmemBytes = kBarBase + kNumBars * 8 + 16 + 1024;
-constexpr uint32_t kTmemCols = 512;      // S/P buffer 0 at col 0, buffer 1 at 128, O at 256
+constexpr uint32_t kTmemCols = 512;      // S/P buffers at columns 0, 128, 256; O at 384
+constexpr uint32_t kOCol = 384;
 constexpr uint32_t kWaitLimit = 1u << 20;
 constexpr float kLog2eF = 1.4426950408889634f;
-
-enum { B_Q = 0, B_KVF = 1, B_KVE = 3, B_SF = 5, B_PF = 7, B_PVD = 9, B_O = 11 };
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
                                               volatile int* abort_flag) {
@@ -69,6 +82,8 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = smem;
+  int32_t* tbl = reinterpret_cast<int32_t*>(smem + kTblOff);
+  float* red = reinterpret_cast<float*>(smem + kRedOff);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarBase);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarBase + kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -76,39 +91,43 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work item: (request, KV head, query tile); heavier (later) tiles first
-  const int nqt = a.max_parts;            // query tiles per request (host: ceil(max_q_len/TQ))
-  int64_t bid = blockIdx.x;
-  const int qt = nqt - 1 - static_cast<int>(bid % nqt);
-  bid /= nqt;
-  const int h = static_cast<int>(bid % a.num_kv_heads);
-  const int r = static_cast<int>(bid / a.num_kv_heads);
+  // ---- work item from the compact list: (request, query tile) x KV head
+  const int item = blockIdx.x / a.num_kv_heads;
+  const int h = blockIdx.x - item * a.num_kv_heads;
+  if (item >= *a.pf_count) return;
+  const int2 rq = a.pf_items[item];
+  const int r = rq.x, qt = rq.y;
   const int cu0 = a.cu_seqlens_q[r];
   const int q_len = a.cu_seqlens_q[r + 1] - cu0;
-  if (q_len < 2 || qt * TQ >= q_len) return;        // decode rows and empty tiles
   const int kv_len = min(a.seqlens_k[r], a.max_context_len);
   const int rows_valid = min(TQ, q_len - qt * TQ);
   const int pos0 = kv_len - q_len + qt * TQ;        // absolute position of tile row 0
   const int last_pos = pos0 + rows_valid - 1;
-  if (last_pos < 0) return;
+  if (rows_valid <= 0 || last_pos < 0) return;
   const int nkv = last_pos / kBN + 1;
   const int n_iter = 2 * nkv;
   const int hq0 = h * G;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars[B_Q], 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars[B_KVF + s], 1);
-      mbar_init(&bars[B_KVE + s], 1);
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(&bars[B_KF + s], kProducerWarps);
+      mbar_init(&bars[B_KE + s], 1);
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(&bars[B_VF + s], kProducerWarps);
+      mbar_init(&bars[B_VE + s], 1);
+    }
+    for (int s = 0; s < kSBufs; ++s) {
       mbar_init(&bars[B_SF + s], 1);
-      mbar_init(&bars[B_PF + s], 128);
+      mbar_init(&bars[B_PF + s], kSoftmaxThreads);
       mbar_init(&bars[B_PVD + s], 1);
     }
     mbar_init(&bars[B_O], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -117,35 +136,41 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
-    // ================================================================ TMA producer
+  if (warp >= kProducerWarp0 && warp < kMmaWarp) {
+    // ================================================================ TMA producers
+    // Producer warp pw loads blocks 2*pw and 2*pw + 1 of every 128-key tile
+    // (both 64-column halves of K, and of V in pass 2) and arms its share of
+    // the tile's expected bytes.
+    const int pw = warp - kProducerWarp0;
+    const int32_t* bt = a.block_tables + static_cast<int64_t>(r) * a.max_blocks_per_seq;
+    const int nblk = last_pos / 16 + 1;               // blocks holding visible keys
+    const int ncache = min(nblk, kTblMax);
+    for (int i = (warp - kProducerWarp0) * 32 + lane; i < ncache; i += kProducerWarps * 32)
+      tbl[i] = __ldg(bt + i);
+    named_bar(2, kProducerWarps * 32);
     if (lane == 0) {
       const int oob_row = a.num_blocks * a.num_kv_heads * 16;
-      const int32_t* bt = a.block_tables + static_cast<int64_t>(r) * a.max_blocks_per_seq;
-      mbar_arrive_expect_tx(&bars[B_Q], kQBytes);
-      tma_load_3d(sQ, &qmap, 0, hq0, cu0 + qt * TQ, &bars[B_Q]);
-      tma_load_3d(sQ + kHalf, &qmap, 64, hq0, cu0 + qt * TQ, &bars[B_Q]);
+      if (pw == 0) {
+        prefetch_tensormap(&kmap);
+        prefetch_tensormap(&vmap);
+        mbar_arrive_expect_tx(&bars[B_Q], kQBytes);
+        tma_load_3d(sQ, &qmap, 0, hq0, cu0 + qt * TQ, &bars[B_Q]);
+        tma_load_3d(sQ + kHalf, &qmap, 64, hq0, cu0 + qt * TQ, &bars[B_Q]);
+      }
       const uint64_t pol = l2_policy_evict_last();
-      uint32_t ph_empty[2] = {0, 0};
-      int issued = 0;
+      constexpr int kBoxesBytes = 2 * 2 * 2048;        // 2 blocks x 2 halves per warp
+      uint32_t ph_ke[kKStages] = {0, 0, 0}, ph_ve[kVStages] = {0, 0};
+      int issued_k = 0, issued_v = 0;
       for (int it = 0; it < n_iter && !*abort_flag; ++it) {
-        const int st = it & 1;
-        if (it >= 2) {
-          if (!wait_or_abort(&bars[B_KVE + st], ph_empty[st], abort_flag)) break;
-          ph_empty[st] ^= 1;
-        }
         const bool pass2 = it >= nkv;
         const int j = pass2 ? it - nkv : it;
-        uint8_t* sK = smem + kQBytes + st * kStageBytes;
-        uint8_t* sV = sK + kKVBytes;
-        mbar_arrive_expect_tx(&bars[B_KVF + st], pass2 ? kStageBytes : kKVBytes);
-        int ys[8];
+        int ys[2];
 #pragma unroll
-        for (int b = 0; b < 8; ++b) {
-          const int key0 = j * kBN + b * 16;
-          int y = oob_row;
-          if (key0 < kv_len) {
-            const int phys = __ldg(bt + key0 / 16);
+        for (int b = 0; b < 2; ++b) {
+          const int blk = j * 8 + 2 * pw + b;
+          int y = oob_row;                                 // past the pool: zero fill
+          if (blk < nblk) {
+            const int phys = blk < kTblMax ? tbl[blk] : __ldg(bt + blk);
             if (static_cast<unsigned>(phys) < static_cast<unsigned>(a.num_blocks))
               y = (phys * a.num_kv_heads + h) * 16;
             else
@@ -153,81 +178,104 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
           }
           ys[b] = y;
         }
-#pragma unroll
-        for (int b = 0; b < 8; ++b) {
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            tma_load_2d(sK + half * kHalf + b * 2048, &kmap, half * 64, ys[b], &bars[B_KVF + st],
-                        pol);
-            if (pass2)
-              tma_load_2d(sV + half * kHalf + b * 2048, &vmap, half * 64, ys[b],
-                          &bars[B_KVF + st], pol);
-          }
+        const int ks = it % kKStages;
+        if (it >= kKStages) {
+          if (!wait_or_abort(&bars[B_KE + ks], ph_ke[ks], abort_flag)) break;
+          ph_ke[ks] ^= 1;
         }
-        issued = it + 1;
+        uint8_t* sK = smem + kKOff + ks * kTileBytes;
+        mbar_arrive_expect_tx(&bars[B_KF + ks], kBoxesBytes);
+#pragma unroll
+        for (int b = 0; b < 2; ++b)
+#pragma unroll
+          for (int half = 0; half < 2; ++half)
+            tma_load_2d(sK + half * kHalf + (2 * pw + b) * 2048, &kmap, half * 64, ys[b],
+                        &bars[B_KF + ks], pol);
+        issued_k = it + 1;
+        if (pass2) {
+          const int vs = j % kVStages;
+          if (j >= kVStages) {
+            if (!wait_or_abort(&bars[B_VE + vs], ph_ve[vs], abort_flag)) break;
+            ph_ve[vs] ^= 1;
+          }
+          uint8_t* sV = smem + kVOff + vs * kTileBytes;
+          mbar_arrive_expect_tx(&bars[B_VF + vs], kBoxesBytes);
+#pragma unroll
+          for (int b = 0; b < 2; ++b)
+#pragma unroll
+            for (int half = 0; half < 2; ++half)
+              tma_load_2d(sV + half * kHalf + (2 * pw + b) * 2048, &vmap, half * 64, ys[b],
+                          &bars[B_VF + vs], pol);
+          issued_v = j + 1;
+        }
       }
       // the last copies into each stage have landed before the CTA may exit
-      for (int it = issued - 1; it >= 0 && it >= issued - 2; --it)
-        (void)mbar_wait_bounded(&bars[B_KVF + (it & 1)], (it >> 1) & 1);
-      (void)mbar_wait_bounded(&bars[B_Q], 0);
+      for (int it = issued_k - 1; it >= 0 && it >= issued_k - kKStages; --it)
+        (void)mbar_wait_bounded(&bars[B_KF + it % kKStages], (it / kKStages) & 1);
+      for (int j = issued_v - 1; j >= 0 && j >= issued_v - kVStages; --j)
+        (void)mbar_wait_bounded(&bars[B_VF + j % kVStages], (j / kVStages) & 1);
+      if (pw == 0) (void)mbar_wait_bounded(&bars[B_Q], 0);
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ================================================================ MMA issuer
     if (lane == 0) {
-      uint32_t ph_full[2] = {0, 0}, ph_pf[2] = {0, 0}, ph_pvd[2] = {0, 0};
+      uint32_t ph_kf[kKStages] = {0, 0, 0}, ph_vf[kVStages] = {0, 0};
+      uint32_t ph_pf[kSBufs] = {0, 0, 0}, ph_pvd[kSBufs] = {0, 0, 0};
       bool ok = wait_or_abort(&bars[B_Q], 0, abort_flag);
       const uint32_t q_addr = smem_u32(sQ);
       bool first_pv = true;
-      auto issue_s = [&](int it) -> bool {
-        const int st = it & 1;
-        if (!wait_or_abort(&bars[B_KVF + st], ph_full[st], abort_flag)) return false;
-        ph_full[st] ^= 1;
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(smem + kQBytes + st * kStageBytes);
-        const uint32_t d = tmem + static_cast<uint32_t>((it & 1) * 128);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t off = (ks >> 2) * kHalf + (ks & 3) * 32;
-          tc_mma_ss(d, smem_desc_sw128(q_addr + off, 16, 1024),
-                    smem_desc_sw128(k_addr + off, 16, 1024), kIdescS, ks > 0 ? 1u : 0u);
-        }
-        tc_commit(&bars[B_SF + (it & 1)]);
-        if (it < nkv) tc_commit(&bars[B_KVE + st]);     // pass 1 only needs K
-        return true;
-      };
-      if (ok) ok = issue_s(0);
+      int next_s = 0;
       for (int it = 0; ok && it < n_iter; ++it) {
-        const int b = it & 1;
-        // S of the next tile into the other buffer, once that buffer is free
-        if (it + 1 < n_iter) {
-          const int pb = (it + 1) & 1;
-          if (it >= 1) {
-            if (it - 1 < nkv) {            // softmax finished reading S(it-1)
-              if (!(ok = wait_or_abort(&bars[B_PF + pb], ph_pf[pb], abort_flag))) break;
-              ph_pf[pb] ^= 1;
-            } else {                       // PV(it-1) finished reading P(it-1)
-              if (!(ok = wait_or_abort(&bars[B_PVD + pb], ph_pvd[pb], abort_flag))) break;
-              ph_pvd[pb] ^= 1;
+        // keep S one tile ahead of PV: reusing the buffer of tile next_s - 3
+        // then waits only for PV(it - 2), while PV(it - 1) stays queued
+        while (ok && next_s < n_iter && next_s <= it + 1) {
+          const int sb = next_s % kSBufs;
+          if (next_s >= kSBufs) {                 // buffer sb held tile next_s - kSBufs
+            const int prev = next_s - kSBufs;
+            if (prev < nkv) {                     // softmax finished reading S(prev)
+              if (!(ok = wait_or_abort(&bars[B_PF + sb], ph_pf[sb], abort_flag))) break;
+              ph_pf[sb] ^= 1;
+            } else {                              // PV(prev) finished reading P(prev)
+              if (!(ok = wait_or_abort(&bars[B_PVD + sb], ph_pvd[sb], abort_flag))) break;
+              ph_pvd[sb] ^= 1;
             }
           }
-          if (!(ok = issue_s(it + 1))) break;
+          const int ks = next_s % kKStages;
+          if (!(ok = wait_or_abort(&bars[B_KF + ks], ph_kf[ks], abort_flag))) break;
+          ph_kf[ks] ^= 1;
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(smem + kKOff + ks * kTileBytes);
+          const uint32_t d = tmem + static_cast<uint32_t>(sb * 128);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
+            tc_mma_ss(d, smem_desc_sw128(q_addr + off, 16, 1024),
+                      smem_desc_sw128(k_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&bars[B_SF + sb]);
+          tc_commit(&bars[B_KE + ks]);            // S is the only reader of K
+          ++next_s;
         }
+        if (!ok) break;
         if (it >= nkv) {
-          // O += P V once the softmax warps have written P(it)
+          // O += P V once the softmax warps have written P(it) and V has landed
+          const int b = it % kSBufs;
           if (!(ok = wait_or_abort(&bars[B_PF + b], ph_pf[b], abort_flag))) break;
           ph_pf[b] ^= 1;
+          const int vs = (it - nkv) % kVStages;
+          if (!(ok = wait_or_abort(&bars[B_VF + vs], ph_vf[vs], abort_flag))) break;
+          ph_vf[vs] ^= 1;
           tc_fence_after();
-          const int st = it & 1;
-          const uint32_t v_addr = smem_u32(smem + kQBytes + st * kStageBytes + kKVBytes);
+          const uint32_t v_addr = smem_u32(smem + kVOff + vs * kTileBytes);
           const uint32_t p_base = tmem + static_cast<uint32_t>(b * 128);
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            const uint64_t vd = smem_desc_sw128(v_addr + ks * 2048, kHalf, 1024);
-            tc_mma_ts(tmem + 256, p_base + ks * 8, vd, kIdescPV, first_pv ? 0u : 1u);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t vd = smem_desc_sw128(v_addr + kk * 2048, kHalf, 1024);
+            tc_mma_ts(tmem + kOCol, p_base + kk * 8, vd, kIdescPV, first_pv ? 0u : 1u);
             first_pv = false;
-            tc_mma_ts(tmem + 256, p_base + 64 + ks * 8, vd, kIdescPV, 1u);
+            tc_mma_ts(tmem + kOCol, p_base + 64 + kk * 8, vd, kIdescPV, 1u);
           }
-          tc_commit(&bars[B_KVE + st]);
+          tc_commit(&bars[B_VE + vs]);
           tc_commit(&bars[B_PVD + b]);
         }
       }
@@ -236,117 +284,139 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
     }
   } else {
     // ================================================================ softmax / epilogue
-    const int t = threadIdx.x;                 // row of the tile == TMEM lane
+    // Warp w owns TMEM lanes 32*(w%4).. (tile rows) and key columns 64*(w/4)..
+    const int quarter = warp & 3, half = warp >> 2;
+    const int t = quarter * 32 + lane;         // tile row == TMEM lane
     const int i = t / G, g = t % G;
     const bool row_ok = i < rows_valid;
     const int pos = pos0 + i;
     const float c = a.scale * kLog2eF;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    float m = -INFINITY, l = 0.f, inv_l = 0.f;
-    uint32_t ph_sf[2] = {0, 0};
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+    uint32_t ph_sf[kSBufs] = {0, 0, 0};
     bool ok = true;
-    for (int it = 0; it < n_iter; ++it) {
-      const int b = it & 1;
+    // -------- pass 1: row maximum of the raw scores (the scale is positive)
+    float m_raw = -INFINITY;
+    for (int it = 0; it < nkv; ++it) {
+      const int b = it % kSBufs;
       if (!wait_or_abort(&bars[B_SF + b], ph_sf[b], abort_flag)) { ok = false; break; }
       ph_sf[b] ^= 1;
       tc_fence_after();
-      const bool pass2 = it >= nkv;
-      const int j = pass2 ? it - nkv : it;
-      uint32_t raw[128];
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        uint32_t (&chunk)[32] = *reinterpret_cast<uint32_t (*)[32]>(raw + 32 * q4);
-        tmem_ld32(lane_base + b * 128 + 32 * q4, chunk);
-      }
+      uint32_t raw[64];
+      tmem_ld32(lane_base + b * 128 + half * 64, *reinterpret_cast<uint32_t (*)[32]>(raw));
+      tmem_ld32(lane_base + b * 128 + half * 64 + 32,
+                *reinterpret_cast<uint32_t (*)[32]>(raw + 32));
       tmem_wait_ld();
-      const int key0 = j * kBN;
-      const int lim = row_ok ? pos - key0 : -1;     // columns n <= lim are visible
-      if (!pass2) {
-        float tm = -INFINITY;
+      const int key0 = it * kBN + half * 64;
+      float mx = -INFINITY;
+      if (it * kBN + kBN - 1 <= pos0) {        // the whole tile is visible to every row
 #pragma unroll
-        for (int n = 0; n < 128; ++n)
-          if (n <= lim) tm = fmaxf(tm, __uint_as_float(raw[n]) * c);
-        const float m_new = fmaxf(m, tm);
-        if (m_new != -INFINITY) {
-          float sum = 0.f;
-#pragma unroll
-          for (int n = 0; n < 128; ++n)
-            if (n <= lim) sum += exp2f(__uint_as_float(raw[n]) * c - m_new);
-          l = l * exp2f(m - m_new) + sum;
-          m = m_new;
-        }
-        tc_fence_before();
-        mbar_arrive(&bars[B_PF + b]);
+        for (int n = 0; n < 64; n += 2)
+          mx = fmax3(mx, __uint_as_float(raw[n]), __uint_as_float(raw[n + 1]));
       } else {
-        if (it == nkv) inv_l = l > 0.f ? 1.f / l : 0.f;
-        uint32_t hi[64], lo[64];
+        const int lim = row_ok ? pos - key0 : -1;
 #pragma unroll
-        for (int n2 = 0; n2 < 64; ++n2) {
-          const int n = 2 * n2;
-          const float p0 = (n <= lim) ? exp2f(__uint_as_float(raw[n]) * c - m) * inv_l : 0.f;
-          const float p1 =
-              (n + 1 <= lim) ? exp2f(__uint_as_float(raw[n + 1]) * c - m) * inv_l : 0.f;
-          const uint32_t hw = pack2<BF16>(p0, p1);
-          hi[n2] = hw;
-          lo[n2] = pack2<BF16>(p0 - lo_half_to_float<BF16>(hw),
-                               p1 - lo_half_to_float<BF16>(hw >> 16));
-        }
-#pragma unroll
-        for (int q2 = 0; q2 < 2; ++q2) {
-          tmem_st32(lane_base + b * 128 + 32 * q2,
-                    *reinterpret_cast<const uint32_t (*)[32]>(hi + 32 * q2));
-          tmem_st32(lane_base + b * 128 + 64 + 32 * q2,
-                    *reinterpret_cast<const uint32_t (*)[32]>(lo + 32 * q2));
-        }
-        // Keys of the context's partial last block that lie past kv_len hold
-        // whatever the slot held; P is 0 there but 0 * NaN is NaN: clear them.
-        const int stale0 = kv_len, stale1 = min((kv_len + 15) & ~15, key0 + kBN);
-        if (stale0 < stale1 && stale0 >= key0) {
-          const int st = it & 1;
-          if (wait_or_abort(&bars[B_KVF + st], (it >> 1) & 1, abort_flag)) {
-            uint8_t* sV = smem + kQBytes + st * kStageBytes + kKVBytes;
-            const int nrows = stale1 - stale0;
-            for (int idx = t; idx < nrows * 16; idx += 128) {
-              const int row = stale0 - key0 + idx / 16;
-              const int c16 = idx % 16;
-              *reinterpret_cast<uint4*>(sV + (c16 >> 3) * kHalf + row * 128 + (c16 & 7) * 16) =
-                  make_uint4(0, 0, 0, 0);
-            }
-            fence_proxy_async_smem();
-          }
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&bars[B_PF + b]);
+        for (int n = 0; n < 64; ++n)
+          if (n <= lim) mx = fmaxf(mx, __uint_as_float(raw[n]));
       }
+      m_raw = fmaxf(m_raw, mx);
+      tc_fence_before();
+      mbar_arrive(&bars[B_PF + b]);
     }
-    // ---- epilogue: O row -> out
+    red[half * 128 + t] = m_raw;
+    named_bar(1, kSoftmaxThreads);
+    const float m_all = fmaxf(red[t], red[128 + t]);
+    const float m = (m_all == -INFINITY) ? 0.f : m_all * c;
+    const uint64_t c2 = f2(c, c), nm2 = f2(-m, -m);
+    uint64_t l2 = f2(0.f, 0.f);
+    // -------- pass 2: unnormalised P = 2^(s*c - m) (hi + lo) and its row sum
+    for (int it = nkv; ok && it < n_iter; ++it) {
+      const int b = it % kSBufs;
+      if (!wait_or_abort(&bars[B_SF + b], ph_sf[b], abort_flag)) { ok = false; break; }
+      ph_sf[b] ^= 1;
+      tc_fence_after();
+      const int j = it - nkv;
+      uint32_t raw[64];
+      tmem_ld32(lane_base + b * 128 + half * 64, *reinterpret_cast<uint32_t (*)[32]>(raw));
+      tmem_ld32(lane_base + b * 128 + half * 64 + 32,
+                *reinterpret_cast<uint32_t (*)[32]>(raw + 32));
+      tmem_wait_ld();
+      const int key0 = j * kBN + half * 64;
+      const bool full = (j * kBN + kBN - 1 <= pos0);
+      const int lim = full ? 63 : (row_ok ? pos - key0 : -1);
+      uint32_t hi[32], lo[32];
+#pragma unroll
+      for (int n2 = 0; n2 < 32; ++n2) {
+        const uint64_t x = ffma2(f2(__uint_as_float(raw[2 * n2]), __uint_as_float(raw[2 * n2 + 1])),
+                                 c2, nm2);
+        float p0 = fast_exp2(f2lo(x)), p1 = fast_exp2(f2hi(x));
+        if (!full) {
+          p0 = (2 * n2 <= lim) ? p0 : 0.f;
+          p1 = (2 * n2 + 1 <= lim) ? p1 : 0.f;
+        }
+        const uint64_t p = f2(p0, p1);
+        l2 = fadd2(l2, p);
+        const uint32_t hw = pack2<BF16>(p0, p1);
+        hi[n2] = hw;
+        const uint64_t r2 = fsub2(p, f2(lo_half_to_float<BF16>(hw), lo_half_to_float<BF16>(hw >> 16)));
+        lo[n2] = pack2<BF16>(f2lo(r2), f2hi(r2));
+      }
+      tmem_st32(lane_base + b * 128 + half * 32, hi);
+      tmem_st32(lane_base + b * 128 + 64 + half * 32, lo);
+      // Keys of the context's partial last block that lie past kv_len hold
+      // whatever the slot held; P is 0 there but 0 * NaN is NaN: clear them.
+      const int tile0 = j * kBN;
+      const int stale0 = kv_len, stale1 = min((kv_len + 15) & ~15, tile0 + kBN);
+      if (stale0 < stale1 && stale0 >= tile0) {
+        const int vs = j % kVStages;
+        if (wait_or_abort(&bars[B_VF + vs], (j / kVStages) & 1, abort_flag)) {
+          uint8_t* sV = smem + kVOff + vs * kTileBytes;
+          const int nrows = stale1 - stale0;
+          const int ts = threadIdx.x;
+          for (int idx = ts; idx < nrows * 16; idx += kSoftmaxThreads) {
+            const int row = stale0 - tile0 + idx / 16;
+            const int c16 = idx % 16;
+            *reinterpret_cast<uint4*>(sV + (c16 >> 3) * kHalf + row * 128 + (c16 & 7) * 16) =
+                make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&bars[B_PF + b]);
+    }
+    // -------- epilogue: O row / l -> out (this warp's 64 of the 128 dims)
+    red[half * 128 + t] = f2lo(l2) + f2hi(l2);
+    named_bar(1, kSoftmaxThreads);
+    const float l_row = red[t] + red[128 + t];
+    const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
     if (ok && wait_or_abort(&bars[B_O], 0, abort_flag)) {
       tc_fence_after();
-      uint32_t o[128];
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4)
-        tmem_ld32(lane_base + 256 + 32 * q4, *reinterpret_cast<uint32_t (*)[32]>(o + 32 * q4));
+      uint32_t o[64];
+      tmem_ld32(lane_base + kOCol + half * 64, *reinterpret_cast<uint32_t (*)[32]>(o));
+      tmem_ld32(lane_base + kOCol + half * 64 + 32, *reinterpret_cast<uint32_t (*)[32]>(o + 32));
       tmem_wait_ld();
       if (row_ok) {
         const int64_t orow =
-            (static_cast<int64_t>(cu0 + qt * TQ + i) * a.num_q_heads + hq0 + g) * 128;
+            (static_cast<int64_t>(cu0 + qt * TQ + i) * a.num_q_heads + hq0 + g) * 128 + half * 64;
         if (a.out_dtype == 3) {
           float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow);
 #pragma unroll
-          for (int k = 0; k < 32; ++k)
-            dst[k] = make_float4(__uint_as_float(o[4 * k]), __uint_as_float(o[4 * k + 1]),
-                                 __uint_as_float(o[4 * k + 2]), __uint_as_float(o[4 * k + 3]));
+          for (int k = 0; k < 16; ++k)
+            dst[k] = make_float4(__uint_as_float(o[4 * k]) * inv_l,
+                                 __uint_as_float(o[4 * k + 1]) * inv_l,
+                                 __uint_as_float(o[4 * k + 2]) * inv_l,
+                                 __uint_as_float(o[4 * k + 3]) * inv_l);
         } else {
           uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + orow);
           const bool ob = (a.out_dtype == 1);
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
+          for (int k = 0; k < 8; ++k) {
             uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float x0 = __uint_as_float(o[8 * k + 2 * e]);
-              const float x1 = __uint_as_float(o[8 * k + 2 * e + 1]);
+              const float x0 = __uint_as_float(o[8 * k + 2 * e]) * inv_l;
+              const float x1 = __uint_as_float(o[8 * k + 2 * e + 1]) * inv_l;
               w[e] = ob ? pack2<true>(x0, x1) : pack2<false>(x0, x1);
             }
             dst[k] = make_uint4(w[0], w[1], w[2], w[3]);
@@ -360,15 +430,49 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
   // given a bounded chance to) before TMEM is released.
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
 }
 
+// Compact list of (request, query tile) items of the q_len >= 2 requests,
+// heaviest tiles of each request first.  One CTA; a block-wide running scan.
+__global__ void __launch_bounds__(256)
+prefill_items_kernel(int32_t num_seqs, const int32_t* cu, int tq, int2* items, int32_t* count,
+                     int32_t capacity) {
+  __shared__ int s_scan[256];
+  __shared__ int s_base;
+  if (threadIdx.x == 0) s_base = 0;
+  __syncthreads();
+  for (int r0 = 0; r0 < num_seqs; r0 += 256) {
+    const int r = r0 + threadIdx.x;
+    int n = 0;
+    if (r < num_seqs) {
+      const int ql = cu[r + 1] - cu[r];
+      n = ql >= 2 ? (ql + tq - 1) / tq : 0;
+    }
+    s_scan[threadIdx.x] = n;
+    __syncthreads();
+    for (int off = 1; off < 256; off <<= 1) {      // inclusive Hillis-Steele scan
+      const int v = threadIdx.x >= off ? s_scan[threadIdx.x - off] : 0;
+      __syncthreads();
+      s_scan[threadIdx.x] += v;
+      __syncthreads();
+    }
+    const int start = s_base + s_scan[threadIdx.x] - n;
+    for (int k = 0; k < n; ++k)
+      if (start + k < capacity) items[start + k] = make_int2(r, n - 1 - k);
+    __syncthreads();
+    if (threadIdx.x == 255) s_base += s_scan[255];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *count = min(s_base, capacity);
+}
+
 template <bool BF16, int G>
 cudaError_t launch_prefill_typed(const AttnArgs& a, const CUtensorMap& k, const CUtensorMap& v,
-                                 const CUtensorMap& q, int nqt, cudaStream_t s) {
+                                 const CUtensorMap& q, int capacity, cudaStream_t s) {
   auto kern = paged_prefill_kernel<BF16, G>;
   static bool configured = false;   // one flag per instantiation
   if (!configured) {
@@ -377,22 +481,20 @@ cudaError_t launch_prefill_typed(const AttnArgs& a, const CUtensorMap& k, const 
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  AttnArgs b = a;
-  b.max_parts = nqt;
-  const int64_t grid = static_cast<int64_t>(a.num_seqs) * a.num_kv_heads * nqt;
+  const int64_t grid = static_cast<int64_t>(capacity) * a.num_kv_heads;
   if (grid == 0) return cudaSuccess;
-  kern<<<static_cast<unsigned>(grid), kPfThreads, kSmemBytes, s>>>(b, k, v, q);
+  kern<<<static_cast<unsigned>(grid), kPfThreads, kSmemBytes, s>>>(a, k, v, q);
   return cudaGetLastError();
 }
 
 template <bool BF16>
 cudaError_t launch_prefill_g(const AttnArgs& a, const CUtensorMap& k, const CUtensorMap& v,
-                             const CUtensorMap& q, int nqt, cudaStream_t s) {
+                             const CUtensorMap& q, int capacity, cudaStream_t s) {
   switch (a.group) {
-    case 1: return launch_prefill_typed<BF16, 1>(a, k, v, q, nqt, s);
-    case 2: return launch_prefill_typed<BF16, 2>(a, k, v, q, nqt, s);
-    case 4: return launch_prefill_typed<BF16, 4>(a, k, v, q, nqt, s);
-    case 8: return launch_prefill_typed<BF16, 8>(a, k, v, q, nqt, s);
+    case 1: return launch_prefill_typed<BF16, 1>(a, k, v, q, capacity, s);
+    case 2: return launch_prefill_typed<BF16, 2>(a, k, v, q, capacity, s);
+    case 4: return launch_prefill_typed<BF16, 4>(a, k, v, q, capacity, s);
+    case 8: return launch_prefill_typed<BF16, 8>(a, k, v, q, capacity, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -407,14 +509,22 @@ bool prefill_supported(int q_dtype, int kv_dtype, int32_t head_dim, int32_t grou
 
 int prefill_query_tile(int32_t group) { return 128 / group; }
 
+int32_t prefill_item_capacity(int32_t num_seqs, int32_t total_q) {
+  // sum_r ceil(q_len_r / tq) over requests with q_len_r >= 2, tq >= 16
+  return total_q / 16 + (num_seqs < total_q / 2 ? num_seqs : total_q / 2) + 1;
+}
+
 cudaError_t launch_paged_prefill(const AttnArgs& a, const CUtensorMap& kmap,
                                  const CUtensorMap& vmap, const CUtensorMap& qmap,
-                                 int32_t max_q_len, cudaStream_t stream) {
+                                 int32_t capacity, cudaStream_t stream) {
   const int tq = 128 / a.group;
-  const int nqt = (max_q_len + tq - 1) / tq;
-  if (nqt <= 0) return cudaSuccess;
-  return a.kv_dtype == 1 ? launch_prefill_g<true>(a, kmap, vmap, qmap, nqt, stream)
-                         : launch_prefill_g<false>(a, kmap, vmap, qmap, nqt, stream);
+  prefill_items_kernel<<<1, 256, 0, stream>>>(a.num_seqs, a.cu_seqlens_q, tq,
+                                              const_cast<int2*>(a.pf_items),
+                                              const_cast<int32_t*>(a.pf_count), capacity);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return a.kv_dtype == 1 ? launch_prefill_g<true>(a, kmap, vmap, qmap, capacity, stream)
+                         : launch_prefill_g<false>(a, kmap, vmap, qmap, capacity, stream);
 }
 
 }  // namespace pa
