@@ -31,7 +31,7 @@ namespace {
 
 constexpr int kSoftmaxWarps = 8;         // two warps per TMEM lane quarter, 64 columns each
 constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
-constexpr int kProducerWarps = 4;        // TMA issue is spread over 4 warps (2 blocks each)
+constexpr int kProducerWarps = 4;        // warps 0-1 of these stream K, 2-3 stream V
 constexpr int kProducerWarp0 = 8;
 constexpr int kMmaWarp = kProducerWarp0 + kProducerWarps;
 constexpr int kPfThreads = (kMmaWarp + 1) * 32;
@@ -111,11 +111,11 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
   if (threadIdx.x == 0) {
     mbar_init(&bars[B_Q], 1);
     for (int s = 0; s < kKStages; ++s) {
-      mbar_init(&bars[B_KF + s], kProducerWarps);
+      mbar_init(&bars[B_KF + s], 2);
       mbar_init(&bars[B_KE + s], 1);
     }
     for (int s = 0; s < kVStages; ++s) {
-      mbar_init(&bars[B_VF + s], kProducerWarps);
+      mbar_init(&bars[B_VF + s], 2);
       mbar_init(&bars[B_VE + s], 1);
     }
     for (int s = 0; s < kSBufs; ++s) {
@@ -138,15 +138,17 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
 
   if (warp >= kProducerWarp0 && warp < kMmaWarp) {
     // ================================================================ TMA producers
-    // Producer warp pw loads blocks 2*pw and 2*pw + 1 of every 128-key tile
-    // (both 64-column halves of K, and of V in pass 2) and arms its share of
-    // the tile's expected bytes.
+    // Two warps stream K tiles (both passes) and two stream V tiles (pass 2),
+    // each loading 4 of the tile's 8 blocks (both 64-column halves) and
+    // arming its share of the expected bytes, so the K ring (3 deep) never
+    // waits behind V.
     const int pw = warp - kProducerWarp0;
+    const bool is_v = pw >= 2;
+    const int sub = pw & 1;                           // blocks 4*sub .. 4*sub+3
     const int32_t* bt = a.block_tables + static_cast<int64_t>(r) * a.max_blocks_per_seq;
     const int nblk = last_pos / 16 + 1;               // blocks holding visible keys
     const int ncache = min(nblk, kTblMax);
-    for (int i = (warp - kProducerWarp0) * 32 + lane; i < ncache; i += kProducerWarps * 32)
-      tbl[i] = __ldg(bt + i);
+    for (int i = pw * 32 + lane; i < ncache; i += kProducerWarps * 32) tbl[i] = __ldg(bt + i);
     named_bar(2, kProducerWarps * 32);
     if (lane == 0) {
       const int oob_row = a.num_blocks * a.num_kv_heads * 16;
@@ -158,16 +160,26 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
         tma_load_3d(sQ + kHalf, &qmap, 64, hq0, cu0 + qt * TQ, &bars[B_Q]);
       }
       const uint64_t pol = l2_policy_evict_last();
-      constexpr int kBoxesBytes = 2 * 2 * 2048;        // 2 blocks x 2 halves per warp
-      uint32_t ph_ke[kKStages] = {0, 0, 0}, ph_ve[kVStages] = {0, 0};
-      int issued_k = 0, issued_v = 0;
-      for (int it = 0; it < n_iter && !*abort_flag; ++it) {
-        const bool pass2 = it >= nkv;
-        const int j = pass2 ? it - nkv : it;
-        int ys[2];
+      constexpr int kShareBytes = 4 * 2 * 2048;        // 4 blocks x 2 halves per warp
+      const int nstage = is_v ? kVStages : kKStages;
+      const int ntiles = is_v ? nkv : n_iter;           // V only in pass 2
+      uint64_t* full = &bars[is_v ? B_VF : B_KF];
+      uint64_t* empty = &bars[is_v ? B_VE : B_KE];
+      const CUtensorMap* map = is_v ? &vmap : &kmap;
+      uint8_t* ring = smem + (is_v ? kVOff : kKOff);
+      uint32_t ph_e[kKStages] = {0, 0, 0};
+      int issued = 0;
+      for (int u = 0; u < ntiles && !*abort_flag; ++u) {
+        const int j = is_v ? u : (u >= nkv ? u - nkv : u);   // key tile
+        const int st = u % nstage;
+        if (u >= nstage) {
+          if (!wait_or_abort(&empty[st], ph_e[st], abort_flag)) break;
+          ph_e[st] ^= 1;
+        }
+        int ys[4];
 #pragma unroll
-        for (int b = 0; b < 2; ++b) {
-          const int blk = j * 8 + 2 * pw + b;
+        for (int b = 0; b < 4; ++b) {
+          const int blk = j * 8 + 4 * sub + b;
           int y = oob_row;                                 // past the pool: zero fill
           if (blk < nblk) {
             const int phys = blk < kTblMax ? tbl[blk] : __ldg(bt + blk);
@@ -178,42 +190,19 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
           }
           ys[b] = y;
         }
-        const int ks = it % kKStages;
-        if (it >= kKStages) {
-          if (!wait_or_abort(&bars[B_KE + ks], ph_ke[ks], abort_flag)) break;
-          ph_ke[ks] ^= 1;
-        }
-        uint8_t* sK = smem + kKOff + ks * kTileBytes;
-        mbar_arrive_expect_tx(&bars[B_KF + ks], kBoxesBytes);
+        uint8_t* dst = ring + st * kTileBytes;
+        mbar_arrive_expect_tx(&full[st], kShareBytes);
 #pragma unroll
-        for (int b = 0; b < 2; ++b)
+        for (int b = 0; b < 4; ++b)
 #pragma unroll
           for (int half = 0; half < 2; ++half)
-            tma_load_2d(sK + half * kHalf + (2 * pw + b) * 2048, &kmap, half * 64, ys[b],
-                        &bars[B_KF + ks], pol);
-        issued_k = it + 1;
-        if (pass2) {
-          const int vs = j % kVStages;
-          if (j >= kVStages) {
-            if (!wait_or_abort(&bars[B_VE + vs], ph_ve[vs], abort_flag)) break;
-            ph_ve[vs] ^= 1;
-          }
-          uint8_t* sV = smem + kVOff + vs * kTileBytes;
-          mbar_arrive_expect_tx(&bars[B_VF + vs], kBoxesBytes);
-#pragma unroll
-          for (int b = 0; b < 2; ++b)
-#pragma unroll
-            for (int half = 0; half < 2; ++half)
-              tma_load_2d(sV + half * kHalf + (2 * pw + b) * 2048, &vmap, half * 64, ys[b],
-                          &bars[B_VF + vs], pol);
-          issued_v = j + 1;
-        }
+            tma_load_2d(dst + half * kHalf + (4 * sub + b) * 2048, map, half * 64, ys[b], &full[st],
+                        pol);
+        issued = u + 1;
       }
       // the last copies into each stage have landed before the CTA may exit
-      for (int it = issued_k - 1; it >= 0 && it >= issued_k - kKStages; --it)
-        (void)mbar_wait_bounded(&bars[B_KF + it % kKStages], (it / kKStages) & 1);
-      for (int j = issued_v - 1; j >= 0 && j >= issued_v - kVStages; --j)
-        (void)mbar_wait_bounded(&bars[B_VF + j % kVStages], (j / kVStages) & 1);
+      for (int u = issued - 1; u >= 0 && u >= issued - nstage; --u)
+        (void)mbar_wait_bounded(&full[u % nstage], (u / nstage) & 1);
       if (pw == 0) (void)mbar_wait_bounded(&bars[B_Q], 0);
     }
   } else if (warp == kMmaWarp) {
