@@ -65,16 +65,20 @@ def peaks():
 
 
 def algorithmic_bytes(W) -> dict:
-    """Bytes the step must move at least once: every visible key and value of
-    every (request, KV head), the queries, the outputs, the block-table
-    entries read, and the new rows written (read + write)."""
-    kv = W.kv_bytes_read()
+    """Bytes the step must move at least once from HBM: every distinct visible
+    K/V slot of every KV head (a block shared by several sequences counts
+    once; it is read from L2 after that), the queries, the outputs, the
+    block-table entries read, and the new rows written (read + write).
+    'kv_logical' counts shared blocks once per sequence (the effective rate)."""
+    kv_logical = W.kv_bytes_read()
+    kv = W.unique_kv_bytes_read()
     q = W.total_q * W.num_q_heads * W.head_dim * 2
     out = W.total_q * W.num_q_heads * W.head_dim * (4 if W.out_dtype == wl.F32 else 2)
     tbl = int((-(-W.seqlens_k.astype(np.int64) // W.block_size)).sum()) * 4 + W.num_seqs * 4
     new = int((W.new_slots >= 0).sum()) * W.num_kv_heads * W.head_dim * 2 * (
         2 + W.kv_elem_bytes()) + W.total_q * 8
-    return {"kv": kv, "attention": kv + q + out + tbl, "step": kv + q + out + tbl + new}
+    return {"kv": kv, "kv_logical": kv_logical, "attention": kv + q + out + tbl,
+            "step": kv + q + out + tbl + new}
 
 
 def workload_name(W) -> str:
@@ -353,7 +357,8 @@ def run_native(args):
             "kv_heads": W.num_kv_heads, "head_dim": W.head_dim, "block_size": W.block_size,
             "num_blocks": W.num_blocks, "mean_context": round(float(W.seqlens_k.mean()), 1),
             "max_context": W.max_context_len, "partition_size": W.partition_size or "auto",
-            "kv_bytes_per_step": by["kv"],
+            "kv_bytes_per_step": by["kv"], "kv_bytes_logical": by["kv_logical"],
+            "effective_gbs": round(by["kv_logical"] * world / (ms * 1e-3) / 1e9, 1),
             "l2": "inputs larger than L2 (KV read per step >> 126 MB); no flush",
             "parallelism": f"replicas x{world}",
         },
@@ -383,17 +388,16 @@ def run_native(args):
 def recorded_traffic(W):
     """DRAM bytes per attention launch from the committed ncu summary, if it
     was taken on this workload with the current kernel source; else None."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
     try:
         with open(path) as f:
-            rec = json.load(f)
-    except (OSError, ValueError):
+            for line in f:
+                parts = line.split()
+                if len(parts) == 3 and parts[0] == W.name and not line.startswith("#"):
+                    return int(parts[2]) if parts[1] == kernel_sha() else None
+    except OSError:
         return None
-    key = W.name
-    entry = rec.get(key)
-    if not entry or entry.get("kernel_sha") != kernel_sha():
-        return None
-    return entry.get("dram_bytes_per_launch")
+    return None
 
 
 def kernel_sha():
