@@ -218,6 +218,43 @@ pa_status pa_decode_static(void* out, pa_dtype out_dtype, const void* q, pa_dtyp
                            int32_t partition_size, void* stream);
 
 /*
+ * Copy whole blocks inside one pool, for copy-on-write ("PagedAttention 与
+ * Continuous Batching", §3.8 COW 与引用计数: when a sequence must append into
+ * a last block still referenced by other sequences, the block manager
+ * allocates a new block, the shared block's contents are copied into it and
+ * the sequence's table is redirected).
+ *
+ * k_cache, v_cache : device pools described by `cache`; block `dst` of both
+ *                receives the contents of block `src` (all heads, all slots).
+ * block_mapping: device int64 [num_pairs][2] = (src, dst) pairs.  A dst must
+ *                not be another pair's src or dst (pairs run concurrently).
+ *                A pair with an id outside [0, num_blocks) is skipped and
+ *                recorded in the device error word.
+ */
+pa_status pa_copy_blocks(void* k_cache, void* v_cache, const pa_cache_desc* cache,
+                         const int64_t* block_mapping, int64_t num_pairs, void* stream);
+
+/*
+ * Move whole blocks between two pools of the same geometry, typically the
+ * device pool and a pinned host pool, for preemption by swapping ("PagedAttention
+ * 与 Continuous Batching", §3.9 Swap 的 IO 代价): block dst of (dst_k, dst_v)
+ * receives block src of (src_k, src_v).
+ *
+ * dst_k, dst_v, src_k, src_v : pool base addresses, device or pinned host
+ *                memory (unified addressing decides the direction).
+ * cache        : geometry (block_size, num_kv_heads, head_dim, kv_dtype);
+ *                its num_blocks is ignored, the two pools' block counts are
+ *                src_num_blocks and dst_num_blocks.
+ * block_mapping: HOST int64 [num_pairs][2] = (src, dst); validated on the host
+ *                (PA_ERR_INVALID_ARG for an id outside its pool).  Runs of
+ *                consecutive pairs are merged into one copy each.
+ */
+pa_status pa_swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
+                         const pa_cache_desc* cache, int64_t src_num_blocks,
+                         int64_t dst_num_blocks, const int64_t* block_mapping, int64_t num_pairs,
+                         void* stream);
+
+/*
  * Read and clear the device error word that kernels set when they skip an
  * out-of-range block id or slot (PA_ERR_OUT_OF_RANGE) or give up a bounded
  * wait (PA_ERR_TIMEOUT).  Synchronises `stream` first.  Returns PA_OK when no

@@ -411,12 +411,16 @@ int oracle_paged_attention(double *out, double *lse, const void *q, int q_dtype,
     if (pair_rows && !pair_heads)
         return OR_BAD_ARG;
 
-    attn_job J = {
-        q, q_dtype, total_q, num_seqs, num_q_heads, cu_seqlens_q, seqlens_k,
-        k_cache, v_cache, num_blocks, block_size, num_kv_heads, head_dim, kv_dtype,
-        k_scale, v_scale, block_tables, max_blocks_per_seq, scale,
-        pair_rows, pair_heads, num_pairs, out, lse, OR_OK,
-    };
+    attn_job J;
+    memset(&J, 0, sizeof J);
+    J.q = q; J.q_dtype = q_dtype; J.total_q = total_q; J.num_seqs = num_seqs;
+    J.num_q_heads = num_q_heads; J.cu_seqlens_q = cu_seqlens_q; J.seqlens_k = seqlens_k;
+    J.k_cache = k_cache; J.v_cache = v_cache; J.num_blocks = num_blocks;
+    J.block_size = block_size; J.num_kv_heads = num_kv_heads; J.head_dim = head_dim;
+    J.kv_dtype = kv_dtype; J.k_scale = k_scale; J.v_scale = v_scale;
+    J.block_tables = block_tables; J.max_blocks_per_seq = max_blocks_per_seq; J.scale = scale;
+    J.pair_rows = pair_rows; J.pair_heads = pair_heads; J.num_pairs = num_pairs;
+    J.out = out; J.lse = lse; J.error = OR_OK;
     pthread_mutex_init(&J.lock, NULL);
     int64_t total = pair_rows ? num_pairs : (int64_t)total_q * num_q_heads;
     int nt = num_threads < 1 ? 1 : num_threads;
@@ -456,4 +460,33 @@ int oracle_paged_attention(double *out, double *lse, const void *q, int q_dtype,
     free(tids);
     pthread_mutex_destroy(&J.lock);
     return J.error;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Whole-block copies (copy-on-write, swap).                                 */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * For each pair (src, dst): block dst of dst_k/dst_v takes the bytes of
+ * block src of src_k/src_v.  A block is block_bytes contiguous bytes
+ * ([num_kv_heads][block_size][head_dim] elements).  Copy-on-write passes the
+ * same pool as source and destination ("PagedAttention 与 Continuous
+ * Batching", §3.8); swapping passes a device-side and a host-side pool (§3.9).
+ */
+int oracle_copy_blocks(void *dst_k, void *dst_v, const void *src_k, const void *src_v,
+                       int64_t src_num_blocks, int64_t dst_num_blocks, int64_t block_bytes,
+                       const int64_t *pairs, int64_t num_pairs)
+{
+    if (!dst_k || !dst_v || !src_k || !src_v || (!pairs && num_pairs) || block_bytes <= 0)
+        return OR_BAD_ARG;
+    for (int64_t i = 0; i < num_pairs; ++i) {
+        int64_t s = pairs[2 * i], d = pairs[2 * i + 1];
+        if (s < 0 || s >= src_num_blocks || d < 0 || d >= dst_num_blocks)
+            return OR_BAD_BLOCK;
+        memmove((char *)dst_k + d * block_bytes, (const char *)src_k + s * block_bytes,
+                (size_t)block_bytes);
+        memmove((char *)dst_v + d * block_bytes, (const char *)src_v + s * block_bytes,
+                (size_t)block_bytes);
+    }
+    return OR_OK;
 }

@@ -55,6 +55,8 @@ def _bind(lib):
         P, P, P, ctypes.c_int, i32, i32, i32, P, P, P, P, i32, i32, i32, i32,
         ctypes.c_int, P, P, P, i32, ctypes.c_double, P, P, i64, ctypes.c_int]
     lib.oracle_paged_attention.restype = ctypes.c_int
+    lib.oracle_copy_blocks.argtypes = [P, P, P, P, i64, i64, i64, P, i64]
+    lib.oracle_copy_blocks.restype = ctypes.c_int
     return lib
 
 
@@ -191,3 +193,17 @@ def paged_decode(q, q_dtype, context_lens, k_cache, v_cache, kv_dtype, block_tab
     cu = np.arange(b + 1, dtype=np.int32)
     return paged_attention(q, q_dtype, cu, context_lens, k_cache, v_cache, kv_dtype,
                            block_tables, scale, **kw)
+
+
+# --- whole-block copies ---------------------------------------------------------
+
+def copy_blocks(dst_k, dst_v, src_k, src_v, pairs):
+    """Block dst of dst_k/dst_v takes block src of src_k/src_v for each
+    (src, dst) row of pairs; pools are [NB, Hkv, BS, D] arrays (in place)."""
+    pairs = _c(np.asarray(pairs).reshape(-1, 2), np.int64)
+    bb = int(np.prod(src_k.shape[1:])) * src_k.itemsize
+    assert dst_k.flags.c_contiguous and src_k.flags.c_contiguous
+    rc = _load().oracle_copy_blocks(_ptr(dst_k), _ptr(dst_v), _ptr(src_k), _ptr(src_v),
+                                    src_k.shape[0], dst_k.shape[0], bb, _ptr(pairs), len(pairs))
+    if rc != 0:
+        raise ValueError(f"oracle_copy_blocks failed: {rc}")

@@ -397,6 +397,67 @@ pa_status pa_varlen(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dty
                        workspace_bytes - head, part_need, s);
 }
 
+static int64_t block_bytes_of(const pa_cache_desc* c) {
+  return static_cast<int64_t>(c->num_kv_heads) * c->block_size * c->head_dim *
+         static_cast<int64_t>(elem_size(c->kv_dtype));
+}
+
+pa_status pa_copy_blocks(void* k_cache, void* v_cache, const pa_cache_desc* cache,
+                         const int64_t* block_mapping, int64_t num_pairs, void* stream) {
+  // geometry only: copying bytes needs no FP8 scales
+  if (!cache || cache->num_blocks <= 0 || cache->num_kv_heads <= 0 || cache->head_dim <= 0 ||
+      cache->block_size <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (!elem_size(cache->kv_dtype) || cache->kv_dtype == PA_F32) return PA_ERR_UNSUPPORTED;
+  if (num_pairs < 0) return PA_ERR_INVALID_ARG;
+  if (num_pairs == 0) return PA_OK;
+  if (!k_cache || !v_cache || !block_mapping) return PA_ERR_INVALID_ARG;
+  const int64_t bb = block_bytes_of(cache);
+  if (bb % 16 != 0 || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(block_mapping, 8))
+    return PA_ERR_INVALID_ARG;
+  cudaError_t e = launch_copy_blocks(k_cache, v_cache, block_mapping, num_pairs, bb,
+                                     cache->num_blocks, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : cuda_fail(e, "copy_blocks launch");
+}
+
+pa_status pa_swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
+                         const pa_cache_desc* cache, int64_t src_num_blocks,
+                         int64_t dst_num_blocks, const int64_t* block_mapping, int64_t num_pairs,
+                         void* stream) {
+  if (!cache || cache->num_kv_heads <= 0 || cache->head_dim <= 0 || cache->block_size <= 0)
+    return PA_ERR_INVALID_ARG;
+  if (!elem_size(cache->kv_dtype) || cache->kv_dtype == PA_F32) return PA_ERR_UNSUPPORTED;
+  if (num_pairs < 0 || src_num_blocks < 0 || dst_num_blocks < 0) return PA_ERR_INVALID_ARG;
+  if (num_pairs == 0) return PA_OK;
+  if (!dst_k || !dst_v || !src_k || !src_v || !block_mapping) return PA_ERR_INVALID_ARG;
+  for (int64_t i = 0; i < num_pairs; ++i) {
+    const int64_t s = block_mapping[2 * i], d = block_mapping[2 * i + 1];
+    if (s < 0 || s >= src_num_blocks || d < 0 || d >= dst_num_blocks) return PA_ERR_INVALID_ARG;
+  }
+  const int64_t bb = block_bytes_of(cache);
+  cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  int64_t i = 0;
+  while (i < num_pairs) {
+    const int64_t s0 = block_mapping[2 * i], d0 = block_mapping[2 * i + 1];
+    int64_t n = 1;
+    while (i + n < num_pairs && block_mapping[2 * (i + n)] == s0 + n &&
+           block_mapping[2 * (i + n) + 1] == d0 + n)
+      ++n;
+    const size_t bytes = static_cast<size_t>(n * bb);
+    cudaError_t e = cudaMemcpyAsync(static_cast<uint8_t*>(dst_k) + d0 * bb,
+                                    static_cast<const uint8_t*>(src_k) + s0 * bb, bytes,
+                                    cudaMemcpyDefault, strm);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(static_cast<uint8_t*>(dst_v) + d0 * bb,
+                          static_cast<const uint8_t*>(src_v) + s0 * bb, bytes, cudaMemcpyDefault,
+                          strm);
+    if (e != cudaSuccess) return cuda_fail(e, "swap_blocks copy");
+    i += n;
+  }
+  return PA_OK;
+}
+
 pa_status pa_device_error(void* stream) {
   cudaError_t e;
   unsigned v = read_and_clear_error_word(static_cast<cudaStream_t>(stream), &e);

@@ -88,6 +88,10 @@ cudaError_t launch_reshape_and_cache(const void* key, const void* value, int src
 
 bool attention_supported(int q_dtype, int kv_dtype, int32_t head_dim, int32_t group);
 
+cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* mapping,
+                               int64_t num_pairs, int64_t block_bytes, int32_t num_blocks,
+                               cudaStream_t stream);
+
 unsigned int read_and_clear_error_word(cudaStream_t stream, cudaError_t* err);
 
 }  // namespace pa

@@ -70,6 +70,10 @@ def load_library(path: str = LIB_PATH):
     lib.pa_varlen.restype = E
     lib.pa_device_error.argtypes = [P]
     lib.pa_device_error.restype = E
+    lib.pa_copy_blocks.argtypes = [P, P, D, P, i64, P]
+    lib.pa_copy_blocks.restype = E
+    lib.pa_swap_blocks.argtypes = [P, P, P, P, D, i64, i64, P, i64, P]
+    lib.pa_swap_blocks.restype = E
     if path == LIB_PATH:
         _lib = lib
     return lib
@@ -208,3 +212,26 @@ def pa_varlen(out: torch.Tensor, q: torch.Tensor, cu_seqlens_q: torch.Tensor,
 def pa_device_error(stream=None) -> int:
     """Read and clear the library's device error word (synchronises the stream)."""
     return int(load_library().pa_device_error(_stream(stream)))
+
+
+def pa_copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, block_mapping: torch.Tensor,
+                   stream=None) -> None:
+    """block_mapping: device int64 [n, 2] of (src, dst) block ids."""
+    desc = cache_desc(k_cache)
+    n = block_mapping.shape[0]
+    st = load_library().pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), ctypes.byref(desc),
+                                       _ptr(block_mapping), n, _stream(stream))
+    _check(st, "pa_copy_blocks")
+
+
+def pa_swap_blocks(dst_k: torch.Tensor, dst_v: torch.Tensor, src_k: torch.Tensor,
+                   src_v: torch.Tensor, block_mapping, stream=None) -> None:
+    """Pools on the device or in pinned host memory; block_mapping: host
+    (src, dst) pairs (anything numpy can turn into int64 [n, 2])."""
+    import numpy as np
+    pairs = np.ascontiguousarray(np.asarray(block_mapping, dtype=np.int64).reshape(-1, 2))
+    desc = cache_desc(src_k)
+    st = load_library().pa_swap_blocks(
+        _ptr(dst_k), _ptr(dst_v), _ptr(src_k), _ptr(src_v), ctypes.byref(desc), src_k.shape[0],
+        dst_k.shape[0], ctypes.c_void_p(pairs.ctypes.data), len(pairs), _stream(stream))
+    _check(st, "pa_swap_blocks")
