@@ -47,6 +47,9 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", type=int, default=2, choices=[2, 3, 4, 5])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--op", default="step", choices=["step", "copy_blocks", "swap_blocks"],
+                    help="step: the attention step (default); copy_blocks / swap_blocks: "
+                         "whole-block copies on the GQA workload's pool geometry")
     ap.add_argument("--batch", type=int, default=None,
                     help="fewer requests, same distributions (profiling captures only)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -498,10 +501,69 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_block_op(args):
+    """Copy-on-write block copies inside the device pool, or swaps between the
+    device pool and a pinned host pool, on Llama-3-8B-shaped blocks (8 KV
+    heads x 16 tokens x 128 dims, bf16: 32 KiB per block per K or V)."""
+    import torch
+    from paged_kv_cache_lens_b200 import pa
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local if world > 1 else 0)
+    rng = np.random.default_rng(77)
+    nb, hkv, bs, d = 16384, 8, 16, 128
+    kc = torch.randn((nb, hkv, bs, d), dtype=torch.bfloat16, device=dev)
+    vc = torch.randn_like(kc)
+    block_bytes = hkv * bs * d * 2
+    stream = torch.cuda.current_stream(dev)
+    if args.op == "copy_blocks":
+        n = 2048                                   # scattered (src, dst) pairs
+        src = rng.choice(nb // 2, n, replace=False)
+        dst = nb // 2 + rng.choice(nb // 2, n, replace=False)
+        mapping = torch.from_numpy(np.stack([src, dst], 1).astype(np.int64)).to(dev)
+        moved = 2 * 2 * n * block_bytes            # K and V, read + write
+        run = lambda: pa.pa_copy_blocks(kc, vc, mapping, stream)  # noqa: E731
+        name = "copy_blocks: HBM GB/s (read + write)"
+        cfg = {"workload": "copy-on-write copies", "pairs": n, "block_bytes": block_bytes}
+    else:
+        n = 512                                    # one 8K-token sequence (page: 512 blocks)
+        hk = torch.empty((n, hkv, bs, d), dtype=torch.bfloat16).pin_memory()
+        hv = torch.empty_like(hk).pin_memory()
+        pairs_out = np.stack([rng.choice(nb, n, replace=False), np.arange(n)], 1)
+        moved = 2 * n * block_bytes                # K and V, one direction
+
+        def run():
+            pa.pa_swap_blocks(hk, hv, kc, vc, pairs_out, stream)
+        name = "swap_blocks: device->host GB/s"
+        cfg = {"workload": "swap out one 8K-token sequence (512 blocks)", "pairs": n,
+               "block_bytes": block_bytes}
+    for _ in range(max(args.warmup, 3)):
+        run()
+    torch.cuda.synchronize(dev)
+    steps = min(args.steps, 200)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    t0.record(stream)
+    for _ in range(steps):
+        run()
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(t0.elapsed_time(t1) / steps, world)
+    assert pa.pa_device_error(stream) == 0
+    if rank == 0:
+        print(json.dumps({"metric": name, "value": round(moved * world / (ms * 1e-3) / 1e9, 1),
+                          "unit": "GB/s", "n_gpus": world, "steps": steps, "warmup": args.warmup,
+                          "ms_per_step": round(ms, 5), "higher_is_better": True,
+                          "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                          "data": "synthetic", "config": cfg, "gpu_launches":
+                          steps if args.op == "copy_blocks" else 0}), flush=True)
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.op != "step":
+        run_block_op(args)
     else:
         run_native(args)
 

@@ -16,7 +16,6 @@ namespace pa {
 
 namespace {
 
-constexpr int kBlockSize = 16;
 constexpr int64_t kAlign = 256;
 
 inline int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
@@ -84,12 +83,12 @@ size_t elem_size(pa_dtype t) {
 pa_status check_cache(const pa_cache_desc* c) {
   if (!c) return PA_ERR_INVALID_ARG;
   if (c->num_blocks <= 0 || c->num_kv_heads <= 0 || c->head_dim <= 0) return PA_ERR_INVALID_ARG;
-  if (c->block_size != kBlockSize) return PA_ERR_UNSUPPORTED;
+  if (c->block_size != 8 && c->block_size != 16 && c->block_size != 32) return PA_ERR_UNSUPPORTED;
   if (c->kv_dtype != PA_F16 && c->kv_dtype != PA_BF16 && c->kv_dtype != PA_FP8_E4M3)
     return PA_ERR_UNSUPPORTED;
   if (c->kv_dtype == PA_FP8_E4M3 && (!c->k_scale || !c->v_scale)) return PA_ERR_INVALID_ARG;
   // TMA row coordinates are 32-bit
-  if (static_cast<int64_t>(c->num_blocks) * c->num_kv_heads * kBlockSize > INT_MAX)
+  if (static_cast<int64_t>(c->num_blocks) * c->num_kv_heads * c->block_size > INT_MAX)
     return PA_ERR_UNSUPPORTED;
   return PA_OK;
 }
@@ -229,7 +228,7 @@ static pa_status check_attention(void* out, pa_dtype out_dtype, const void* q, p
   if (!out || !q || !k_cache || !v_cache || !block_tables) return PA_ERR_INVALID_ARG;
   if (num_q_heads <= 0 || num_q_heads % cache->num_kv_heads != 0) return PA_ERR_INVALID_ARG;
   if (max_context_len < 0 || max_blocks_per_seq < 0) return PA_ERR_INVALID_ARG;
-  if (cdiv(max_context_len, kBlockSize) > max_blocks_per_seq) return PA_ERR_INVALID_ARG;
+  if (cdiv(max_context_len, cache->block_size) > max_blocks_per_seq) return PA_ERR_INVALID_ARG;
   if (out_dtype != PA_F16 && out_dtype != PA_BF16 && out_dtype != PA_F32)
     return PA_ERR_UNSUPPORTED;
   const int32_t group = num_q_heads / cache->num_kv_heads;
@@ -259,12 +258,13 @@ static pa_status run_attention(AttnArgs& a, const pa_cache_desc* cache, int32_t 
     a.ws_m = a.ws_l = a.ws_o = nullptr;
   }
   const int64_t pool_rows = static_cast<int64_t>(cache->num_blocks) * cache->num_kv_heads *
-                            kBlockSize;
+                            cache->block_size;
+  const int32_t box_rows = cache->block_size < 16 ? cache->block_size : 16;
   CUtensorMap kmap, vmap;
   if (!make_pool_tensor_map(&kmap, a.k_cache, cache->kv_dtype, pool_rows, cache->head_dim,
-                            kBlockSize) ||
+                            box_rows) ||
       !make_pool_tensor_map(&vmap, a.v_cache, cache->kv_dtype, pool_rows, cache->head_dim,
-                            kBlockSize))
+                            box_rows))
     return map_fail("the KV pool");
   cudaError_t e = launch_paged_attention(a, kmap, vmap, stream);
   return e == cudaSuccess ? PA_OK : cuda_fail(e, "attention launch");
@@ -365,12 +365,13 @@ pa_status pa_varlen(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dty
     // q_len >= 2 requests: the tensor-core prefill over a compact work list;
     // q_len == 1 requests: the decode kernel, one work row per request.
     const int64_t pool_rows =
-        static_cast<int64_t>(cache->num_blocks) * cache->num_kv_heads * kBlockSize;
+        static_cast<int64_t>(cache->num_blocks) * cache->num_kv_heads * cache->block_size;
+    const int32_t box_rows = cache->block_size < 16 ? cache->block_size : 16;
     CUtensorMap kmap, vmap, qmap;
     if (!make_pool_tensor_map(&kmap, k_cache, cache->kv_dtype, pool_rows, cache->head_dim,
-                              kBlockSize) ||
+                              box_rows) ||
         !make_pool_tensor_map(&vmap, v_cache, cache->kv_dtype, pool_rows, cache->head_dim,
-                              kBlockSize) ||
+                              box_rows) ||
         !make_q_tensor_map(&qmap, q, total_q, num_q_heads, cache->head_dim, group,
                            prefill_query_tile(group)))
       return map_fail("the prefill operands");

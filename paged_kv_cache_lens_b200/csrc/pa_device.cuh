@@ -336,4 +336,36 @@ __device__ __host__ __forceinline__ constexpr uint32_t idesc_f16(bool bf16, int 
          | (static_cast<uint32_t>(M >> 4) << 24);      // M >> 4
 }
 
+// The pool rows (TMA row coordinates) holding 16-token tile `tile` of a run of
+// blocks whose ids start at tbl[0]: one box of 16 rows for 16- and 32-token
+// blocks, two boxes of 8 rows (y1, the second half of the tile) for 8-token
+// blocks.  `nblk` blocks of the run hold data; a second 8-token block past
+// them is read from row `oob_row` (past the pool: zero filled).  Returns
+// false if a block id the tile needs lies outside the pool.
+__device__ __forceinline__ bool tile_rows(const int32_t* tbl, int tile, int bs, int nblk,
+                                          int num_blocks, int hkv, int h, int oob_row, int& y0,
+                                          int& y1) {
+  y1 = -1;
+  if (bs == 16) {
+    const int p = tbl[tile];
+    if (static_cast<unsigned>(p) >= static_cast<unsigned>(num_blocks)) return false;
+    y0 = (p * hkv + h) * 16;
+  } else if (bs == 32) {
+    const int p = tbl[tile >> 1];
+    if (static_cast<unsigned>(p) >= static_cast<unsigned>(num_blocks)) return false;
+    y0 = (p * hkv + h) * 32 + 16 * (tile & 1);
+  } else {
+    const int p0 = tbl[2 * tile];
+    if (static_cast<unsigned>(p0) >= static_cast<unsigned>(num_blocks)) return false;
+    y0 = (p0 * hkv + h) * 8;
+    y1 = oob_row;
+    if (2 * tile + 1 < nblk) {
+      const int p1 = tbl[2 * tile + 1];
+      if (static_cast<unsigned>(p1) >= static_cast<unsigned>(num_blocks)) return false;
+      y1 = (p1 * hkv + h) * 8;
+    }
+  }
+  return true;
+}
+
 }  // namespace pa

@@ -38,7 +38,7 @@ namespace {
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr int kBlockTokens = 16;
-constexpr int kMaxPartitionBlocks = 64;   // partition_size <= 1024 tokens
+constexpr int kMaxPartitionBlocks = 128;  // partition_size <= 1024 tokens, blocks >= 8 tokens
 constexpr float kLog2e = 1.4426950408889634f;
 
 enum { KV_F16 = 0, KV_BF16 = 1, KV_FP8 = 2 };
@@ -143,11 +143,13 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
   if (part >= nparts) return;
   const int tok0 = part * PS;
   const int ntok = min(PS, L - tok0);
-  const int nblk = (ntok + kBlockTokens - 1) / kBlockTokens;
+  const int nblk = (ntok + kBlockTokens - 1) / kBlockTokens;   // 16-token tiles
+  const int bs = a.block_size;
+  const int npblk = (ntok + bs - 1) / bs;                          // pool blocks
 
   const int32_t* bt = a.block_tables + static_cast<int64_t>(seq) * a.max_blocks_per_seq +
-                      tok0 / kBlockTokens;
-  for (int i = threadIdx.x; i < nblk; i += kThreads) tbl[i] = bt[i];
+                      tok0 / bs;
+  for (int i = threadIdx.x; i < npblk; i += kThreads) tbl[i] = bt[i];
   if (threadIdx.x == 0) {
     for (int i = 0; i < kWarps * NSTAGE; ++i) mbar_init(&bars[i], 1);
     fence_barrier_init();
@@ -162,23 +164,27 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
   const uint64_t policy = l2_policy_evict_first();
   const int num_blocks = a.num_blocks;
 
+  const int oob_row = num_blocks * a.num_kv_heads * bs;
   auto issue = [&](int k) {
     const int i = warp + k * kWarps;
     const int s = k % NSTAGE;
-    const int phys = tbl[i];
     uint64_t* bar = wb + s;
-    if (static_cast<unsigned>(phys) >= static_cast<unsigned>(num_blocks)) {
+    int y0, y1;
+    if (!tile_rows(tbl, i, bs, npblk, num_blocks, a.num_kv_heads, h, oob_row, y0, y1)) {
       report_error(kErrBlockRange);
       mbar_arrive(bar);
       return;
     }
     mbar_arrive_expect_tx(bar, 2 * kTB);
-    const int y = (phys * a.num_kv_heads + h) * kBlockTokens;
     uint8_t* kt = wt + s * 2 * kTB;
 #pragma unroll
     for (int b = 0; b < G::kBoxes; ++b) {
-      tma_load_2d(kt + b * G::kBoxBytes, &kmap, b * G::kBoxElems, y, bar, policy);
-      tma_load_2d(kt + kTB + b * G::kBoxBytes, &vmap, b * G::kBoxElems, y, bar, policy);
+      tma_load_2d(kt + b * G::kBoxBytes, &kmap, b * G::kBoxElems, y0, bar, policy);
+      tma_load_2d(kt + kTB + b * G::kBoxBytes, &vmap, b * G::kBoxElems, y0, bar, policy);
+      if (y1 >= 0) {          // 8-token blocks: rows 8..15 of the tile from the next block
+        tma_load_2d(kt + b * G::kBoxBytes + 1024, &kmap, b * G::kBoxElems, y1, bar, policy);
+        tma_load_2d(kt + kTB + b * G::kBoxBytes + 1024, &vmap, b * G::kBoxElems, y1, bar, policy);
+      }
     }
   };
   if (lane == 0)
@@ -256,8 +262,9 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
       dead = true;
       break;
     }
-    const int phys = tbl[i];
-    const bool valid_blk = static_cast<unsigned>(phys) < static_cast<unsigned>(num_blocks);
+    int y0_, y1_;
+    const bool valid_blk =
+        tile_rows(tbl, i, bs, npblk, num_blocks, a.num_kv_heads, h, oob_row, y0_, y1_);
     const int valid = valid_blk ? min(kBlockTokens, ntok - i * kBlockTokens) : 0;
     const uint8_t* kt = wt + s * 2 * kTB;
     const uint8_t* vt = kt + kTB;

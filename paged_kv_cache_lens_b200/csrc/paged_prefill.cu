@@ -146,12 +146,13 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
     const bool is_v = pw >= 2;
     const int sub = pw & 1;                           // blocks 4*sub .. 4*sub+3
     const int32_t* bt = a.block_tables + static_cast<int64_t>(r) * a.max_blocks_per_seq;
-    const int nblk = last_pos / 16 + 1;               // blocks holding visible keys
+    const int bs = a.block_size;
+    const int nblk = last_pos / bs + 1;               // blocks holding visible keys
     const int ncache = min(nblk, kTblMax);
     for (int i = pw * 32 + lane; i < ncache; i += kProducerWarps * 32) tbl[i] = __ldg(bt + i);
     named_bar(2, kProducerWarps * 32);
     if (lane == 0) {
-      const int oob_row = a.num_blocks * a.num_kv_heads * 16;
+      const int oob_row = a.num_blocks * a.num_kv_heads * bs;
       if (pw == 0) {
         prefetch_tensormap(&kmap);
         prefetch_tensormap(&vmap);
@@ -176,28 +177,36 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
           if (!wait_or_abort(&empty[st], ph_e[st], abort_flag)) break;
           ph_e[st] ^= 1;
         }
-        int ys[4];
+        // this warp's four 16-key sub-tiles of key tile j (one box of 16 rows,
+        // or two of 8 rows for 8-token blocks); past the visible keys the box
+        // starts past the pool and is zero filled
+        int ys[4], ys1[4];
 #pragma unroll
         for (int b = 0; b < 4; ++b) {
-          const int blk = j * 8 + 4 * sub + b;
-          int y = oob_row;                                 // past the pool: zero fill
-          if (blk < nblk) {
-            const int phys = blk < kTblMax ? tbl[blk] : __ldg(bt + blk);
-            if (static_cast<unsigned>(phys) < static_cast<unsigned>(a.num_blocks))
-              y = (phys * a.num_kv_heads + h) * 16;
-            else
+          const int sti = j * 8 + 4 * sub + b;
+          ys[b] = oob_row;
+          ys1[b] = bs == 8 ? oob_row : -1;
+          if (sti * 16 <= last_pos) {
+            const int32_t* src = (sti + 1) * 16 / bs + 1 < kTblMax ? tbl : bt;
+            int y0, y1;
+            if (tile_rows(src, sti, bs, nblk, a.num_blocks, a.num_kv_heads, h, oob_row, y0, y1)) {
+              ys[b] = y0;
+              ys1[b] = y1;
+            } else {
               report_error(kErrBlockRange);
+            }
           }
-          ys[b] = y;
         }
         uint8_t* dst = ring + st * kTileBytes;
         mbar_arrive_expect_tx(&full[st], kShareBytes);
 #pragma unroll
         for (int b = 0; b < 4; ++b)
 #pragma unroll
-          for (int half = 0; half < 2; ++half)
-            tma_load_2d(dst + half * kHalf + (4 * sub + b) * 2048, map, half * 64, ys[b], &full[st],
-                        pol);
+          for (int half = 0; half < 2; ++half) {
+            uint8_t* box = dst + half * kHalf + (4 * sub + b) * 2048;
+            tma_load_2d(box, map, half * 64, ys[b], &full[st], pol);
+            if (ys1[b] >= 0) tma_load_2d(box + 1024, map, half * 64, ys1[b], &full[st], pol);
+          }
         issued = u + 1;
       }
       // the last copies into each stage have landed before the CTA may exit

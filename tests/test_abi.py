@@ -76,8 +76,8 @@ def test_host_validation_rejects_before_any_launch(lib):
     # null output
     assert lib.pa_decode(None, 0, fake, 0, 4, 2, fake, fake, ctypes.byref(desc), fake, 8, fake,
                          100, 0.125, 0, None, 0, None) == 1
-    # block size other than 16
-    bad = _desc(block_size=32)
+    # block size other than 8, 16 or 32
+    bad = _desc(block_size=64)
     assert lib.pa_decode(fake, 0, fake, 0, 4, 2, fake, fake, ctypes.byref(bad), fake, 8, fake,
                          100, 0.125, 0, None, 0, None) == 2
     # table too narrow for max_context_len

@@ -40,9 +40,10 @@ def _run_small(oracle, W, out_dtype=F32, partition_size=None):
 # ---------------------------------------------------------------- cache write
 
 @pytest.mark.parametrize("kv", [wl.BF16, wl.F16, wl.FP8_E4M3])
-def test_reshape_and_cache_bit_exact(oracle, kv):
+@pytest.mark.parametrize("bs", [8, 16, 32])
+def test_reshape_and_cache_bit_exact(oracle, kv, bs):
     W = wl.build_workload("rc", 101, [1, 1, 1, 7], [1, 30, 64, 100], 8, 4, 128,
-                          dtype=wl.F16 if kv == wl.F16 else wl.BF16, kv_dtype=kv)
+                          dtype=wl.F16 if kv == wl.F16 else wl.BF16, kv_dtype=kv, block_size=bs)
     W.new_slots[2] = -1                          # a padding token is skipped
     d = DeviceStep(W)
     d.fill_cache()
@@ -88,6 +89,34 @@ def test_decode_edge_lengths(oracle, hq, hkv, D):
                           hkv, D, dtype=wl.BF16)
     for ps in (0, 64, 512):
         _run_small(oracle, W, F32, partition_size=ps)
+
+
+@pytest.mark.parametrize("bs", [8, 32])
+@pytest.mark.parametrize("hq,hkv,D", [(4, 4, 64), (8, 2, 128), (16, 2, 256)])
+def test_decode_block_sizes(oracle, bs, hq, hkv, D):
+    """8- and 32-token blocks ("PagedAttention 与 Continuous Batching", §3.7
+    block_size 的取舍: 8, 16 or 32), with edge lengths around both sizes."""
+    lens = [1, 7, 8, 9, 31, 32, 33, 100, 511, 513]
+    W = wl.build_workload("bs", 500 + bs + D, np.ones(len(lens), np.int64), lens, hq, hkv, D,
+                          block_size=bs)
+    for ps in (0, 64):
+        _run_small(oracle, W, F32, partition_size=ps)
+
+
+@pytest.mark.parametrize("bs", [8, 32])
+def test_decode_fp8_block_sizes(oracle, bs):
+    W = wl.build_workload("bs8", 510 + bs, np.ones(4, np.int64), [5, 40, 700, 1111], 8, 2, 128,
+                          kv_dtype=wl.FP8_E4M3, block_size=bs)
+    _run_small(oracle, W, F32)
+
+
+@pytest.mark.parametrize("bs", [8, 32])
+def test_varlen_block_sizes(oracle, bs):
+    q_lens = [1, 130, 1, 257, 33]
+    kv_lens = [77, 130 + 45, 999, 257 + 300, 33]
+    for hq, hkv in [(32, 8), (4, 4)]:
+        W = wl.build_workload("vbs", 520 + bs + hq, q_lens, kv_lens, hq, hkv, 128, block_size=bs)
+        _run_small(oracle, W, F32)
 
 
 @pytest.mark.parametrize("D", [128, 256])
