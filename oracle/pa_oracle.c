@@ -238,6 +238,8 @@ typedef struct {
     const int32_t *block_tables; int32_t max_blocks_per_seq;
     double scale;
     const int64_t *pair_rows; const int32_t *pair_heads; int64_t num_pairs;
+    int32_t window;                  /* > 0: keys pos-window+1 .. pos only */
+    const float *alibi_slopes;       /* [num_q_heads] or NULL */
     double *out; double *lse;
     int error;               /* first error seen by any worker */
     pthread_mutex_t lock;
@@ -281,13 +283,21 @@ static int attend_one(const attn_job *J, int64_t row, int32_t hq, double *out, d
     int64_t n = last + 1 < kv_len ? last + 1 : kv_len;
     if (n < 0)
         n = 0;
+    /* sliding window: only the `window` most recent keys up to the query's
+     * own position are visible */
+    int64_t first = 0;
+    if (J->window > 0 && last - J->window + 1 > 0)
+        first = last - J->window + 1;
+    if (first > n)
+        first = n;
     int32_t h = hq / (J->num_q_heads / J->num_kv_heads);
+    double slope = J->alibi_slopes ? (double)J->alibi_slopes[hq] : 0.0;
 
     for (int32_t d = 0; d < D; ++d)
         out[d] = 0.0;
     if (lse)
         *lse = -INFINITY;
-    if (n == 0)
+    if (n == 0 || first >= n)
         return OR_OK;
 
     double *qv = (double *)malloc(sizeof(double) * D);
@@ -300,8 +310,8 @@ static int attend_one(const attn_job *J, int64_t row, int32_t hq, double *out, d
         qv[d] = load_as_double(J->q, (row * J->num_q_heads + hq) * (int64_t)D + d, J->q_dtype);
 
     int rc = OR_OK;
-    /* pass 1: scores s_t = scale * <q, k_t> */
-    for (int64_t t = 0; t < n && rc == OR_OK; ++t) {
+    /* pass 1: scores s_t = scale * <q, k_t> (+ ALiBi bias slope * (t - pos)) */
+    for (int64_t t = first; t < n && rc == OR_OK; ++t) {
         double dot = 0.0;
         for (int32_t d = 0; d < D; ++d) {
             double k;
@@ -310,20 +320,20 @@ static int attend_one(const attn_job *J, int64_t row, int32_t hq, double *out, d
                 break;
             dot += qv[d] * k;
         }
-        s[t] = J->scale * dot;
+        s[t] = J->scale * dot + slope * (double)(t - last);
     }
     if (rc == OR_OK) {
-        double m = s[0];
-        for (int64_t t = 1; t < n; ++t)
+        double m = s[first];
+        for (int64_t t = first + 1; t < n; ++t)
             if (s[t] > m)
                 m = s[t];
         double denom = 0.0;
-        for (int64_t t = 0; t < n; ++t) {
+        for (int64_t t = first; t < n; ++t) {
             s[t] = exp(s[t] - m);              /* s now holds the weights */
             denom += s[t];
         }
         /* pass 2: out = sum_t w_t v_t / sum_t w_t */
-        for (int64_t t = 0; t < n && rc == OR_OK; ++t) {
+        for (int64_t t = first; t < n && rc == OR_OK; ++t) {
             for (int32_t d = 0; d < D; ++d) {
                 double v;
                 rc = cached(J, J->v_cache, J->v_scale, r, h, t, d, &v);
@@ -389,15 +399,16 @@ static void *attn_worker(void *arg)
  * num_threads: worker threads over independent pairs (<= 1: the caller's).
  * Decode is the special case cu_seqlens_q = 0,1,..,B and seqlens_k = context_lens.
  */
-int oracle_paged_attention(double *out, double *lse, const void *q, int q_dtype,
-                           int32_t total_q, int32_t num_seqs, int32_t num_q_heads,
-                           const int32_t *cu_seqlens_q, const int32_t *seqlens_k,
-                           const void *k_cache, const void *v_cache, int32_t num_blocks,
-                           int32_t block_size, int32_t num_kv_heads, int32_t head_dim,
-                           int kv_dtype, const float *k_scale, const float *v_scale,
-                           const int32_t *block_tables, int32_t max_blocks_per_seq,
-                           double scale, const int64_t *pair_rows, const int32_t *pair_heads,
-                           int64_t num_pairs, int num_threads)
+int oracle_paged_attention_ex(double *out, double *lse, const void *q, int q_dtype,
+                              int32_t total_q, int32_t num_seqs, int32_t num_q_heads,
+                              const int32_t *cu_seqlens_q, const int32_t *seqlens_k,
+                              const void *k_cache, const void *v_cache, int32_t num_blocks,
+                              int32_t block_size, int32_t num_kv_heads, int32_t head_dim,
+                              int kv_dtype, const float *k_scale, const float *v_scale,
+                              const int32_t *block_tables, int32_t max_blocks_per_seq,
+                              double scale, const int64_t *pair_rows, const int32_t *pair_heads,
+                              int64_t num_pairs, int num_threads, int32_t window,
+                              const float *alibi_slopes)
 {
     if (!out || !q || !cu_seqlens_q || !seqlens_k || !k_cache || !v_cache || !block_tables)
         return OR_BAD_ARG;
@@ -420,6 +431,7 @@ int oracle_paged_attention(double *out, double *lse, const void *q, int q_dtype,
     J.kv_dtype = kv_dtype; J.k_scale = k_scale; J.v_scale = v_scale;
     J.block_tables = block_tables; J.max_blocks_per_seq = max_blocks_per_seq; J.scale = scale;
     J.pair_rows = pair_rows; J.pair_heads = pair_heads; J.num_pairs = num_pairs;
+    J.window = window; J.alibi_slopes = alibi_slopes;
     J.out = out; J.lse = lse; J.error = OR_OK;
     pthread_mutex_init(&J.lock, NULL);
     int64_t total = pair_rows ? num_pairs : (int64_t)total_q * num_q_heads;
@@ -460,6 +472,24 @@ int oracle_paged_attention(double *out, double *lse, const void *q, int q_dtype,
     free(tids);
     pthread_mutex_destroy(&J.lock);
     return J.error;
+}
+
+/* Plain attention (no window, no ALiBi): the definition the pages give. */
+int oracle_paged_attention(double *out, double *lse, const void *q, int q_dtype,
+                           int32_t total_q, int32_t num_seqs, int32_t num_q_heads,
+                           const int32_t *cu_seqlens_q, const int32_t *seqlens_k,
+                           const void *k_cache, const void *v_cache, int32_t num_blocks,
+                           int32_t block_size, int32_t num_kv_heads, int32_t head_dim,
+                           int kv_dtype, const float *k_scale, const float *v_scale,
+                           const int32_t *block_tables, int32_t max_blocks_per_seq,
+                           double scale, const int64_t *pair_rows, const int32_t *pair_heads,
+                           int64_t num_pairs, int num_threads)
+{
+    return oracle_paged_attention_ex(out, lse, q, q_dtype, total_q, num_seqs, num_q_heads,
+                                     cu_seqlens_q, seqlens_k, k_cache, v_cache, num_blocks,
+                                     block_size, num_kv_heads, head_dim, kv_dtype, k_scale,
+                                     v_scale, block_tables, max_blocks_per_seq, scale,
+                                     pair_rows, pair_heads, num_pairs, num_threads, 0, NULL);
 }
 
 /* ------------------------------------------------------------------------ */

@@ -55,6 +55,9 @@ def _bind(lib):
         P, P, P, ctypes.c_int, i32, i32, i32, P, P, P, P, i32, i32, i32, i32,
         ctypes.c_int, P, P, P, i32, ctypes.c_double, P, P, i64, ctypes.c_int]
     lib.oracle_paged_attention.restype = ctypes.c_int
+    lib.oracle_paged_attention_ex.argtypes = lib.oracle_paged_attention.argtypes + [
+        ctypes.c_int32, P]
+    lib.oracle_paged_attention_ex.restype = ctypes.c_int
     lib.oracle_copy_blocks.argtypes = [P, P, P, P, i64, i64, i64, P, i64]
     lib.oracle_copy_blocks.restype = ctypes.c_int
     return lib
@@ -149,7 +152,7 @@ def reshape_and_cache(key, value, src_dtype, slot_mapping, k_cache, v_cache, blo
 
 def paged_attention(q, q_dtype, cu_seqlens_q, seqlens_k, k_cache, v_cache, kv_dtype,
                     block_tables, scale, k_scale=None, v_scale=None, pairs=None,
-                    with_lse=False, num_threads=1):
+                    with_lse=False, num_threads=1, window=0, alibi_slopes=None):
     """fp64 attention over the paged cache.
 
     q: [total_q, Hq, D] (bit patterns).  pairs: optional (rows, heads) arrays;
@@ -176,11 +179,12 @@ def paged_attention(q, q_dtype, cu_seqlens_q, seqlens_k, k_cache, v_cache, kv_dt
         npairs = len(prow)
         out = np.empty((npairs, d), np.float64)
         lse = np.empty((npairs,), np.float64) if with_lse else None
-    rc = _load().oracle_paged_attention(
+    slopes = _c(alibi_slopes, np.float32)
+    rc = _load().oracle_paged_attention_ex(
         _ptr(out), _ptr(lse), _ptr(q), q_dtype, total_q, len(sk), hq, _ptr(cu), _ptr(sk),
         _ptr(np.ascontiguousarray(k_cache)), _ptr(np.ascontiguousarray(v_cache)), nb, bs, hkv, d,
         kv_dtype, _ptr(ks), _ptr(vs), _ptr(bt), bt.shape[1], float(scale), _ptr(prow),
-        _ptr(phead), npairs, int(num_threads))
+        _ptr(phead), npairs, int(num_threads), int(window), _ptr(slopes))
     if rc != 0:
         raise ValueError(f"oracle_paged_attention failed: {rc}")
     return (out, lse) if with_lse else out

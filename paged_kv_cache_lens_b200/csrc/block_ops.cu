@@ -55,7 +55,49 @@ copy_blocks_kernel(uint8_t* k_cache, uint8_t* v_cache, const int64_t* __restrict
   }
 }
 
+// Gather/scatter of whole blocks between two pools that may live in device
+// memory or in device-mapped pinned host memory: one CTA per pair and pool,
+// 16-byte accesses; over the host link the many independent requests in
+// flight keep it busy where one copy per scattered block would not.  The
+// (src, dst) pairs travel by value in the kernel parameters (up to
+// kMovePairs per launch), so the host-side mapping needs no device copy.
+__global__ void __launch_bounds__(kCopyThreads)
+move_blocks_kernel(uint8_t* dst_k, uint8_t* dst_v, const uint8_t* src_k, const uint8_t* src_v,
+                   const __grid_constant__ MovePairs pairs, int64_t block_bytes) {
+  const int pair = blockIdx.x >> 1;
+  const bool v = blockIdx.x & 1;
+  const int64_t src = pairs.p[2 * pair], dst = pairs.p[2 * pair + 1];
+  const uint4* s = reinterpret_cast<const uint4*>((v ? src_v : src_k) + src * block_bytes);
+  uint4* d = reinterpret_cast<uint4*>((v ? dst_v : dst_k) + dst * block_bytes);
+  const int64_t n16 = block_bytes / 16;
+  for (int64_t i = threadIdx.x; i < n16; i += 4 * kCopyThreads) {
+    uint4 r[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (i + u * kCopyThreads < n16) r[u] = s[i + u * kCopyThreads];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (i + u * kCopyThreads < n16) d[i + u * kCopyThreads] = r[u];
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_move_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
+                               const int64_t* host_mapping, int64_t num_pairs,
+                               int64_t block_bytes, cudaStream_t stream) {
+  for (int64_t s0 = 0; s0 < num_pairs; s0 += kMovePairs) {
+    MovePairs mp;
+    const int64_t n = min(static_cast<int64_t>(kMovePairs), num_pairs - s0);
+    for (int64_t i = 0; i < 2 * n; ++i) mp.p[i] = host_mapping[2 * s0 + i];
+    move_blocks_kernel<<<static_cast<unsigned>(2 * n), kCopyThreads, 0, stream>>>(
+        static_cast<uint8_t*>(dst_k), static_cast<uint8_t*>(dst_v),
+        static_cast<const uint8_t*>(src_k), static_cast<const uint8_t*>(src_v), mp, block_bytes);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
 
 cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* mapping,
                                int64_t num_pairs, int64_t block_bytes, int32_t num_blocks,

@@ -438,6 +438,24 @@ pa_status pa_swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void
   }
   const int64_t bb = block_bytes_of(cache);
   cudaStream_t strm = static_cast<cudaStream_t>(stream);
+  // Pools the GPU can address (device memory, mapped pinned host memory):
+  // one gather/scatter kernel per 1024 pairs.  Otherwise one copy per run.
+  auto addressable = [](const void* p) {
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return false;
+    }
+    return at.type == cudaMemoryTypeDevice ||
+           (at.type == cudaMemoryTypeHost && at.devicePointer == p);
+  };
+  if (bb % 16 == 0 && addressable(dst_k) && addressable(dst_v) && addressable(src_k) &&
+      addressable(src_v) && aligned(dst_k, 16) && aligned(dst_v, 16) && aligned(src_k, 16) &&
+      aligned(src_v, 16)) {
+    cudaError_t e =
+        launch_move_blocks(dst_k, dst_v, src_k, src_v, block_mapping, num_pairs, bb, strm);
+    return e == cudaSuccess ? PA_OK : cuda_fail(e, "swap_blocks launch");
+  }
   int64_t i = 0;
   while (i < num_pairs) {
     const int64_t s0 = block_mapping[2 * i], d0 = block_mapping[2 * i + 1];

@@ -88,6 +88,16 @@ cudaError_t launch_reshape_and_cache(const void* key, const void* value, int src
 
 bool attention_supported(int q_dtype, int kv_dtype, int32_t head_dim, int32_t group);
 
+// (src, dst) block pairs passed by value to one launch (16 KiB of parameters).
+constexpr int kMovePairs = 1024;
+struct MovePairs {
+  int64_t p[2 * kMovePairs];
+};
+// Whole-block moves between two device-accessible pools (device memory or
+// mapped pinned host memory); the mapping is read on the host.
+cudaError_t launch_move_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
+                               const int64_t* host_mapping, int64_t num_pairs,
+                               int64_t block_bytes, cudaStream_t stream);
 cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* mapping,
                                int64_t num_pairs, int64_t block_bytes, int32_t num_blocks,
                                cudaStream_t stream);

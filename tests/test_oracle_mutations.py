@@ -16,7 +16,7 @@ from tests._helpers import oracle_attention, oracle_pools
 SRC = os.path.join(os.path.dirname(pa_oracle.__file__), "pa_oracle.c")
 
 MUTATIONS = {
-    "drop_logit_scale": ("s[t] = J->scale * dot;", "s[t] = dot;"),
+    "drop_logit_scale": ("s[t] = J->scale * dot + slope", "s[t] = dot + slope"),
     "causal_off_by_one": ("int64_t last = kv_len - q_len + i;", "int64_t last = kv_len - q_len + i - 1;"),
     "top_left_causal": ("int64_t last = kv_len - q_len + i;", "int64_t last = i;"),
     "gqa_interleaved": ("int32_t h = hq / (J->num_q_heads / J->num_kv_heads);",
@@ -27,6 +27,8 @@ MUTATIONS = {
                             "int64_t dst = ((blk * num_kv_heads + h) * block_size + (block_size - 1 - off)) * head_dim + d;"),
     "fp8_ties_away": ("    return fmod(n, 2.0) == 0.0 ? n : n + 1.0;", "    return n + 1.0;"),
     "fp8_scale_multiplied": ("*v *= (double)sc[h];", "*v /= (double)sc[h];"),
+    "window_off_by_one": ("first = last - J->window + 1;", "first = last - J->window;"),
+    "alibi_sign": ("slope * (double)(t - last)", "slope * (double)(last - t)"),
     "table_row_stride": ("J->block_tables[(int64_t)r * J->max_blocks_per_seq + t / J->block_size]",
                          "J->block_tables[(int64_t)r * (J->max_blocks_per_seq - 1) + t / J->block_size]"),
 }
@@ -81,6 +83,13 @@ def _pins_pass(orc) -> bool:
             out = oracle_attention(orc, W, kc, vc)
             if not np.allclose(out, _sdpa(W, kt, vt), rtol=0, atol=1e-12):
                 return False
+        from tests.test_oracle_options import _reference
+        W = wl.build_workload("mo", 32, [1, 6, 20], [40, 6, 52], 4, 2, 16)
+        kc, vc = oracle_pools(orc, W)
+        sl = np.array([0.5, 0.25, 0.125, 0.0625], np.float32)
+        got = oracle_attention(orc, W, kc, vc, window=11, alibi_slopes=sl)
+        if not np.allclose(got, _reference(W, kc, vc, window=11, slopes=sl), rtol=0, atol=1e-12):
+            return False
         return True
     except (ValueError, IndexError):
         return False
