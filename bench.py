@@ -52,6 +52,9 @@ def parse_args():
                          "whole-block copies on the GQA workload's pool geometry")
     ap.add_argument("--batch", type=int, default=None,
                     help="fewer requests, same distributions (profiling captures only)")
+    ap.add_argument("--window", type=int, default=0,
+                    help="sliding window (keys per query) for the attention variant")
+    ap.add_argument("--alibi", action="store_true", help="ALiBi slopes 2^(-8 i / H)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -244,13 +247,18 @@ def run_native(args):
                                           W.max_context_len)
     ws = torch.empty(max(nws, 256), dtype=torch.uint8, device=dev)
 
+    slopes = None
+    if args.alibi:
+        slopes = torch.tensor([2.0 ** (-8.0 * (i + 1) / W.num_q_heads)
+                               for i in range(W.num_q_heads)], dtype=torch.float32, device=dev)
+
     def attend(q_, bt_, sk_, cu_, out_):
         if W.decode:
             pa.pa_decode(out_, q_, kc, vc, bt_, sk_, W.max_context_len, W.scale, ks, vs,
-                         W.partition_size, ws, stream)
+                         W.partition_size, ws, stream, window=args.window, alibi_slopes=slopes)
         else:
             pa.pa_varlen(out_, q_, cu_, sk_, W.max_q_len, W.max_context_len, kc, vc, bt_,
-                         W.scale, ks, vs, ws, stream)
+                         W.scale, ks, vs, ws, stream, window=args.window, alibi_slopes=slopes)
 
     def step():
         pa.pa_reshape_and_cache(nk, nv, slots, kc, vc, ks, vs, stream)
@@ -364,6 +372,7 @@ def run_native(args):
             "effective_gbs": round(by["kv_logical"] * world / (ms * 1e-3) / 1e9, 1),
             "l2": "inputs larger than L2 (KV read per step >> 126 MB); no flush",
             "parallelism": f"replicas x{world}",
+            "window": args.window, "alibi": bool(args.alibi),
         },
         "roofline": {
             "bound": "hbm", "kernel": "pa_decode" if W.decode else "pa_varlen",

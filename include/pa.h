@@ -155,6 +155,30 @@ pa_status pa_decode(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dty
                     void* stream);
 
 /*
+ * Optional attention variants ("PagedAttention 与 Continuous Batching", §10.8
+ * FAQ: paged kernels must also cover sliding window and ALiBi).  A zeroed
+ * struct (or a NULL pointer) means plain attention.
+ */
+typedef struct {
+    int32_t window;              /* > 0: a query at absolute position p sees only
+                                    keys p - window + 1 .. p; <= 0: no window */
+    const float* alibi_slopes;   /* NULL, or device fp32 [num_q_heads]: adds
+                                    slope[hq] * (key position - query position)
+                                    to the scaled logit (a non-positive bias) */
+} pa_attn_options;
+
+/*
+ * pa_decode with options (NULL = pa_decode).
+ */
+pa_status pa_decode_ex(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dtype,
+                       int32_t batch, int32_t num_q_heads, const void* k_cache,
+                       const void* v_cache, const pa_cache_desc* cache,
+                       const int32_t* block_tables, int32_t max_blocks_per_seq,
+                       const int32_t* context_lens, int32_t max_context_len, float scale,
+                       int32_t partition_size, const pa_attn_options* options, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/*
  * Bytes of workspace pa_varlen needs for these sizes.
  */
 size_t pa_varlen_workspace_size(int32_t num_seqs, int32_t total_q, int32_t num_q_heads,
@@ -253,6 +277,17 @@ pa_status pa_swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void
                          const pa_cache_desc* cache, int64_t src_num_blocks,
                          int64_t dst_num_blocks, const int64_t* block_mapping, int64_t num_pairs,
                          void* stream);
+
+/*
+ * pa_varlen with options (NULL = pa_varlen).
+ */
+pa_status pa_varlen_ex(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dtype,
+                       int32_t total_q, int32_t num_seqs, int32_t num_q_heads,
+                       const int32_t* cu_seqlens_q, const int32_t* seqlens_k, int32_t max_q_len,
+                       int32_t max_context_len, const void* k_cache, const void* v_cache,
+                       const pa_cache_desc* cache, const int32_t* block_tables,
+                       int32_t max_blocks_per_seq, float scale, const pa_attn_options* options,
+                       void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Read and clear the device error word that kernels set when they skip an

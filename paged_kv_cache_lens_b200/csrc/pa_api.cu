@@ -295,6 +295,16 @@ static void fill_common(AttnArgs& a, void* out, pa_dtype out_dtype, const void* 
   a.v_cache = v_cache;
 }
 
+static pa_status apply_options(AttnArgs& a, const pa_attn_options* o) {
+  a.window = 0;
+  a.alibi = nullptr;
+  if (!o) return PA_OK;
+  if (o->alibi_slopes && !aligned(o->alibi_slopes, 4)) return PA_ERR_INVALID_ARG;
+  a.window = o->window > 0 ? o->window : 0;
+  a.alibi = o->alibi_slopes;
+  return PA_OK;
+}
+
 pa_status pa_decode(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dtype,
                     int32_t batch, int32_t num_q_heads, const void* k_cache,
                     const void* v_cache, const pa_cache_desc* cache,
@@ -302,6 +312,18 @@ pa_status pa_decode(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dty
                     const int32_t* context_lens, int32_t max_context_len, float scale,
                     int32_t partition_size, void* workspace, size_t workspace_bytes,
                     void* stream) {
+  return pa_decode_ex(out, out_dtype, q, q_dtype, batch, num_q_heads, k_cache, v_cache, cache,
+                      block_tables, max_blocks_per_seq, context_lens, max_context_len, scale,
+                      partition_size, nullptr, workspace, workspace_bytes, stream);
+}
+
+pa_status pa_decode_ex(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dtype,
+                       int32_t batch, int32_t num_q_heads, const void* k_cache,
+                       const void* v_cache, const pa_cache_desc* cache,
+                       const int32_t* block_tables, int32_t max_blocks_per_seq,
+                       const int32_t* context_lens, int32_t max_context_len, float scale,
+                       int32_t partition_size, const pa_attn_options* options, void* workspace,
+                       size_t workspace_bytes, void* stream) {
   if (batch < 0) return PA_ERR_INVALID_ARG;
   pa_status st = check_attention(out, out_dtype, q, q_dtype, num_q_heads, k_cache, v_cache,
                                  cache, block_tables, max_blocks_per_seq, max_context_len);
@@ -315,6 +337,8 @@ pa_status pa_decode(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dty
   a.rows = batch;
   a.num_seqs = batch;
   a.context_lens = context_lens;
+  st = apply_options(a, options);
+  if (st != PA_OK) return st;
   const int32_t ps = resolve_partition(batch, num_q_heads, max_context_len, partition_size);
   const size_t need =
       pa_decode_workspace_size(batch, num_q_heads, cache->head_dim, max_context_len, ps);
@@ -329,6 +353,19 @@ pa_status pa_varlen(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dty
                     const pa_cache_desc* cache, const int32_t* block_tables,
                     int32_t max_blocks_per_seq, float scale, void* workspace,
                     size_t workspace_bytes, void* stream) {
+  return pa_varlen_ex(out, out_dtype, q, q_dtype, total_q, num_seqs, num_q_heads, cu_seqlens_q,
+                      seqlens_k, max_q_len, max_context_len, k_cache, v_cache, cache,
+                      block_tables, max_blocks_per_seq, scale, nullptr, workspace,
+                      workspace_bytes, stream);
+}
+
+pa_status pa_varlen_ex(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dtype,
+                       int32_t total_q, int32_t num_seqs, int32_t num_q_heads,
+                       const int32_t* cu_seqlens_q, const int32_t* seqlens_k, int32_t max_q_len,
+                       int32_t max_context_len, const void* k_cache, const void* v_cache,
+                       const pa_cache_desc* cache, const int32_t* block_tables,
+                       int32_t max_blocks_per_seq, float scale, const pa_attn_options* options,
+                       void* workspace, size_t workspace_bytes, void* stream) {
   if (total_q < 0 || num_seqs < 0 || max_q_len < 0) return PA_ERR_INVALID_ARG;
   pa_status st = check_attention(out, out_dtype, q, q_dtype, num_q_heads, k_cache, v_cache,
                                  cache, block_tables, max_blocks_per_seq, max_context_len);
@@ -353,11 +390,13 @@ pa_status pa_varlen(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dty
   const size_t head = static_cast<size_t>(2 * map_bytes + item_bytes);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int32_t group = num_q_heads / cache->num_kv_heads;
-  const bool chunks = max_q_len >= 2 && scale > 0.f && aligned(out, 16) &&
+  const bool chunks = max_q_len >= 2 && aligned(out, 16) &&
                       prefill_supported(q_dtype, cache->kv_dtype, cache->head_dim, group);
   AttnArgs a;
   fill_common(a, out, out_dtype, q, q_dtype, num_q_heads, k_cache, v_cache, cache, block_tables,
               max_blocks_per_seq, scale);
+  st = apply_options(a, options);
+  if (st != PA_OK) return st;
   a.num_seqs = num_seqs;
   a.cu_seqlens_q = cu_seqlens_q;
   a.seqlens_k = seqlens_k;

@@ -34,6 +34,8 @@ struct AttnArgs {
   const float* v_scale;
   float scale;
   int32_t max_context_len;      // host bound; longer rows are clamped to it
+  int32_t window;               // > 0: a query at position p sees keys p-window+1 .. p
+  const float* alibi;           // [Hq] ALiBi slopes (bias slope * (key - p)) or nullptr
   int32_t partition_size;       // tokens per split-K partition
   int32_t max_parts;            // partitions of the longest row
   float* ws_m;                  // [rows][Hq][max_parts] running max (log2 domain)

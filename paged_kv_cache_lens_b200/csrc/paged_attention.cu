@@ -143,6 +143,10 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
   if (part >= nparts) return;
   const int tok0 = part * PS;
   const int ntok = min(PS, L - tok0);
+  // sliding window: visible keys are lo .. L-1 (the query sits at L-1)
+  const int lo = a.window > 0 ? max(0, L - a.window) : 0;
+  const int t_lo = max(0, lo - tok0);                  // first visible token of the partition
+  const int first_tile = t_lo / kBlockTokens;
   const int nblk = (ntok + kBlockTokens - 1) / kBlockTokens;   // 16-token tiles
   const int bs = a.block_size;
   const int npblk = (ntok + bs - 1) / bs;                          // pool blocks
@@ -160,13 +164,14 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
   uint8_t* wt = tiles + warp * NSTAGE * 2 * kTB;
   uint64_t* wb = bars + warp * NSTAGE;
   uint16_t* pt = pt_all + warp * kNT * 8 * kBlockTokens;
-  const int my_blocks = nblk > warp ? (nblk - warp + kWarps - 1) / kWarps : 0;
+  const int ntiles = nblk - first_tile;                // tiles holding visible keys
+  const int my_blocks = ntiles > warp ? (ntiles - warp + kWarps - 1) / kWarps : 0;
   const uint64_t policy = l2_policy_evict_first();
   const int num_blocks = a.num_blocks;
 
   const int oob_row = num_blocks * a.num_kv_heads * bs;
   auto issue = [&](int k) {
-    const int i = warp + k * kWarps;
+    const int i = first_tile + warp + k * kWarps;
     const int s = k % NSTAGE;
     uint64_t* bar = wb + s;
     int y0, y1;
@@ -237,6 +242,15 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
     qk_mul *= a.k_scale[h];
     v_mul = a.v_scale[h];
   }
+  // ALiBi slopes of this lane's two score columns (query heads hq0 + 2c + j),
+  // in the log2 domain; the bias of key t is slope * (t - (L - 1))
+  float alibi[2] = {0.f, 0.f};
+  if (a.alibi) {
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+      if (2 * c + j < group && 2 * c + j < GT) alibi[j] = a.alibi[hq0 + 2 * c + j] * kLog2e;
+  }
+  const int key_base = tok0 - (L - 1);                 // key position - query position
 
   // ---- online-softmax state (columns 2c, 2c+1 of this lane) and output
   float m_run[2] = {-INFINITY, -INFINITY};
@@ -252,7 +266,7 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
   bool dead = false;
   int k = 0;
   for (; k < my_blocks; ++k) {
-    const int i = warp + k * kWarps;
+    const int i = first_tile + warp + k * kWarps;
     const int s = k % NSTAGE;
     const uint32_t parity = (k / NSTAGE) & 1;
     bool ok = mbar_wait_bounded(wb + s, parity);
@@ -322,7 +336,11 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int t = r + ((e >> 1) << 3);
-        sv[e] = (t < valid) ? (sacc[0][e] + sacc[1][e]) * qk_mul : -INFINITY;
+        const int trel = i * kBlockTokens + t;         // token within the partition
+        sv[e] = (t < valid && trel >= t_lo)
+                    ? (sacc[0][e] + sacc[1][e]) * qk_mul +
+                          alibi[e & 1] * static_cast<float>(key_base + trel)
+                    : -INFINITY;
       }
       float alpha[2], pv[4];
 #pragma unroll

@@ -105,7 +105,11 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
   const int last_pos = pos0 + rows_valid - 1;
   if (rows_valid <= 0 || last_pos < 0) return;
   const int nkv = last_pos / kBN + 1;
-  const int n_iter = 2 * nkv;
+  // sliding window: key tiles before the first key any row of the tile sees
+  // are skipped (tiles jlo .. nkv-1 are visited, ntile of them)
+  const int jlo = a.window > 0 ? max(0, pos0 - a.window + 1) / kBN : 0;
+  const int ntile = nkv - jlo;
+  const int n_iter = 2 * ntile;
   const int hq0 = h * G;
 
   if (threadIdx.x == 0) {
@@ -163,7 +167,7 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
       const uint64_t pol = l2_policy_evict_last();
       constexpr int kShareBytes = 4 * 2 * 2048;        // 4 blocks x 2 halves per warp
       const int nstage = is_v ? kVStages : kKStages;
-      const int ntiles = is_v ? nkv : n_iter;           // V only in pass 2
+      const int ntiles = is_v ? ntile : n_iter;         // V only in pass 2
       uint64_t* full = &bars[is_v ? B_VF : B_KF];
       uint64_t* empty = &bars[is_v ? B_VE : B_KE];
       const CUtensorMap* map = is_v ? &vmap : &kmap;
@@ -171,7 +175,7 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
       uint32_t ph_e[kKStages] = {0, 0, 0};
       int issued = 0;
       for (int u = 0; u < ntiles && !*abort_flag; ++u) {
-        const int j = is_v ? u : (u >= nkv ? u - nkv : u);   // key tile
+        const int j = jlo + (is_v ? u : (u >= ntile ? u - ntile : u));   // key tile
         const int st = u % nstage;
         if (u >= nstage) {
           if (!wait_or_abort(&empty[st], ph_e[st], abort_flag)) break;
@@ -230,7 +234,7 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
           const int sb = next_s % kSBufs;
           if (next_s >= kSBufs) {                 // buffer sb held tile next_s - kSBufs
             const int prev = next_s - kSBufs;
-            if (prev < nkv) {                     // softmax finished reading S(prev)
+            if (prev < ntile) {                   // softmax finished reading S(prev)
               if (!(ok = wait_or_abort(&bars[B_PF + sb], ph_pf[sb], abort_flag))) break;
               ph_pf[sb] ^= 1;
             } else {                              // PV(prev) finished reading P(prev)
@@ -255,12 +259,12 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
           ++next_s;
         }
         if (!ok) break;
-        if (it >= nkv) {
+        if (it >= ntile) {
           // O += P V once the softmax warps have written P(it) and V has landed
           const int b = it % kSBufs;
           if (!(ok = wait_or_abort(&bars[B_PF + b], ph_pf[b], abort_flag))) break;
           ph_pf[b] ^= 1;
-          const int vs = (it - nkv) % kVStages;
+          const int vs = (it - ntile) % kVStages;
           if (!(ok = wait_or_abort(&bars[B_VF + vs], ph_vf[vs], abort_flag))) break;
           ph_vf[vs] ^= 1;
           tc_fence_after();
@@ -292,64 +296,81 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     uint32_t ph_sf[kSBufs] = {0, 0, 0};
     bool ok = true;
-    // -------- pass 1: row maximum of the raw scores (the scale is positive)
-    float m_raw = -INFINITY;
-    for (int it = 0; it < nkv; ++it) {
+    // Row visibility: keys lo_row .. pos (lo_row from the sliding window);
+    // logits in the log2 domain x = s*scale*log2e + slope*log2e*(key - pos).
+    const int lo_row = a.window > 0 ? pos - a.window + 1 : 0;
+    const float slope = a.alibi ? a.alibi[hq0 + g] * kLog2eF : 0.f;
+    const uint64_t c2 = f2(c, c);
+    // a tile every row sees in full needs no mask
+    auto tile_full = [&](int j) {
+      return j * kBN + kBN - 1 <= pos0 && (a.window <= 0 || j * kBN >= last_pos - a.window + 1);
+    };
+    // -------- pass 1: row maximum of the logits
+    float m_x = -INFINITY;
+    for (int it = 0; it < ntile; ++it) {
       const int b = it % kSBufs;
       if (!wait_or_abort(&bars[B_SF + b], ph_sf[b], abort_flag)) { ok = false; break; }
       ph_sf[b] ^= 1;
       tc_fence_after();
-      uint32_t raw[64];
-      tmem_ld32(lane_base + b * 128 + half * 64, *reinterpret_cast<uint32_t (*)[32]>(raw));
-      tmem_ld32(lane_base + b * 128 + half * 64 + 32,
-                *reinterpret_cast<uint32_t (*)[32]>(raw + 32));
-      tmem_wait_ld();
-      const int key0 = it * kBN + half * 64;
-      float mx = -INFINITY;
-      if (it * kBN + kBN - 1 <= pos0) {        // the whole tile is visible to every row
-#pragma unroll
-        for (int n = 0; n < 64; n += 2)
-          mx = fmax3(mx, __uint_as_float(raw[n]), __uint_as_float(raw[n + 1]));
-      } else {
-        const int lim = row_ok ? pos - key0 : -1;
-#pragma unroll
-        for (int n = 0; n < 64; ++n)
-          if (n <= lim) mx = fmaxf(mx, __uint_as_float(raw[n]));
-      }
-      m_raw = fmaxf(m_raw, mx);
-      tc_fence_before();
-      mbar_arrive(&bars[B_PF + b]);
-    }
-    red[half * 128 + t] = m_raw;
-    named_bar(1, kSoftmaxThreads);
-    const float m_all = fmaxf(red[t], red[128 + t]);
-    const float m = (m_all == -INFINITY) ? 0.f : m_all * c;
-    const uint64_t c2 = f2(c, c), nm2 = f2(-m, -m);
-    uint64_t l2 = f2(0.f, 0.f);
-    // -------- pass 2: unnormalised P = 2^(s*c - m) (hi + lo) and its row sum
-    for (int it = nkv; ok && it < n_iter; ++it) {
-      const int b = it % kSBufs;
-      if (!wait_or_abort(&bars[B_SF + b], ph_sf[b], abort_flag)) { ok = false; break; }
-      ph_sf[b] ^= 1;
-      tc_fence_after();
-      const int j = it - nkv;
+      const int j = jlo + it;
       uint32_t raw[64];
       tmem_ld32(lane_base + b * 128 + half * 64, *reinterpret_cast<uint32_t (*)[32]>(raw));
       tmem_ld32(lane_base + b * 128 + half * 64 + 32,
                 *reinterpret_cast<uint32_t (*)[32]>(raw + 32));
       tmem_wait_ld();
       const int key0 = j * kBN + half * 64;
-      const bool full = (j * kBN + kBN - 1 <= pos0);
-      const int lim = full ? 63 : (row_ok ? pos - key0 : -1);
+      const float b0 = slope * static_cast<float>(key0 - pos);
+      float mx = -INFINITY;
+      if (tile_full(j)) {
+#pragma unroll
+        for (int n2 = 0; n2 < 32; ++n2) {
+          const uint64_t x = ffma2(f2(__uint_as_float(raw[2 * n2]), __uint_as_float(raw[2 * n2 + 1])),
+                                   c2, f2(b0 + slope * (2 * n2), b0 + slope * (2 * n2 + 1)));
+          mx = fmax3(mx, f2lo(x), f2hi(x));
+        }
+      } else {
+        const int nlo = row_ok ? lo_row - key0 : 64, nhi = row_ok ? pos - key0 : -1;
+#pragma unroll
+        for (int n = 0; n < 64; ++n)
+          if (n >= nlo && n <= nhi)
+            mx = fmaxf(mx, fmaf(__uint_as_float(raw[n]), c, b0 + slope * n));
+      }
+      m_x = fmaxf(m_x, mx);
+      tc_fence_before();
+      mbar_arrive(&bars[B_PF + b]);
+    }
+    red[half * 128 + t] = m_x;
+    named_bar(1, kSoftmaxThreads);
+    const float m_all = fmaxf(red[t], red[128 + t]);
+    const float m = (m_all == -INFINITY) ? 0.f : m_all;
+    uint64_t l2 = f2(0.f, 0.f);
+    // -------- pass 2: unnormalised P = 2^(x - m) (hi + lo) and its row sum
+    for (int it = ntile; ok && it < n_iter; ++it) {
+      const int b = it % kSBufs;
+      if (!wait_or_abort(&bars[B_SF + b], ph_sf[b], abort_flag)) { ok = false; break; }
+      ph_sf[b] ^= 1;
+      tc_fence_after();
+      const int vi = it - ntile;                 // position in the V ring sequence
+      const int j = jlo + vi;
+      uint32_t raw[64];
+      tmem_ld32(lane_base + b * 128 + half * 64, *reinterpret_cast<uint32_t (*)[32]>(raw));
+      tmem_ld32(lane_base + b * 128 + half * 64 + 32,
+                *reinterpret_cast<uint32_t (*)[32]>(raw + 32));
+      tmem_wait_ld();
+      const int key0 = j * kBN + half * 64;
+      const bool full = tile_full(j);
+      const int nlo = full ? 0 : (row_ok ? lo_row - key0 : 64);
+      const int nhi = full ? 63 : (row_ok ? pos - key0 : -1);
+      const float b0 = slope * static_cast<float>(key0 - pos) - m;
       uint32_t hi[32], lo[32];
 #pragma unroll
       for (int n2 = 0; n2 < 32; ++n2) {
         const uint64_t x = ffma2(f2(__uint_as_float(raw[2 * n2]), __uint_as_float(raw[2 * n2 + 1])),
-                                 c2, nm2);
+                                 c2, f2(b0 + slope * (2 * n2), b0 + slope * (2 * n2 + 1)));
         float p0 = fast_exp2(f2lo(x)), p1 = fast_exp2(f2hi(x));
         if (!full) {
-          p0 = (2 * n2 <= lim) ? p0 : 0.f;
-          p1 = (2 * n2 + 1 <= lim) ? p1 : 0.f;
+          p0 = (2 * n2 >= nlo && 2 * n2 <= nhi) ? p0 : 0.f;
+          p1 = (2 * n2 + 1 >= nlo && 2 * n2 + 1 <= nhi) ? p1 : 0.f;
         }
         const uint64_t p = f2(p0, p1);
         l2 = fadd2(l2, p);
@@ -365,8 +386,8 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
       const int tile0 = j * kBN;
       const int stale0 = kv_len, stale1 = min((kv_len + 15) & ~15, tile0 + kBN);
       if (stale0 < stale1 && stale0 >= tile0) {
-        const int vs = j % kVStages;
-        if (wait_or_abort(&bars[B_VF + vs], (j / kVStages) & 1, abort_flag)) {
+        const int vs = vi % kVStages;
+        if (wait_or_abort(&bars[B_VF + vs], (vi / kVStages) & 1, abort_flag)) {
           uint8_t* sV = smem + kVOff + vs * kTileBytes;
           const int nrows = stale1 - stale0;
           const int ts = threadIdx.x;

@@ -34,6 +34,10 @@ class PaError(RuntimeError):
         super().__init__(f"{where}: {pa_status_string(status)}")
 
 
+class pa_attn_options(ctypes.Structure):
+    _fields_ = [("window", ctypes.c_int32), ("alibi_slopes", ctypes.c_void_p)]
+
+
 class pa_cache_desc(ctypes.Structure):
     _fields_ = [("num_blocks", ctypes.c_int32), ("block_size", ctypes.c_int32),
                 ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
@@ -70,6 +74,13 @@ def load_library(path: str = LIB_PATH):
     lib.pa_varlen.restype = E
     lib.pa_device_error.argtypes = [P]
     lib.pa_device_error.restype = E
+    O = ctypes.POINTER(pa_attn_options)
+    lib.pa_decode_ex.argtypes = [P, E, P, E, i32, i32, P, P, D, P, i32, P, i32, F, i32, O, P, sz,
+                                 P]
+    lib.pa_decode_ex.restype = E
+    lib.pa_varlen_ex.argtypes = [P, E, P, E, i32, i32, i32, P, P, i32, i32, P, P, D, P, i32, F, O,
+                                 P, sz, P]
+    lib.pa_varlen_ex.restype = E
     lib.pa_copy_blocks.argtypes = [P, P, D, P, i64, P]
     lib.pa_copy_blocks.restype = E
     lib.pa_swap_blocks.argtypes = [P, P, P, P, D, i64, i64, P, i64, P]
@@ -171,42 +182,62 @@ def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]):
     return workspace, workspace.numel() * workspace.element_size()
 
 
+def _options(window: int, alibi_slopes: Optional[torch.Tensor]):
+    if not window and alibi_slopes is None:
+        return None
+    return ctypes.byref(pa_attn_options(int(window or 0), _ptr(alibi_slopes).value
+                                        if alibi_slopes is not None else None))
+
+
 def pa_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
               block_tables: torch.Tensor, context_lens: torch.Tensor, max_context_len: int,
               scale: float, k_scale=None, v_scale=None, partition_size: int = 0,
-              workspace: Optional[torch.Tensor] = None, stream=None) -> None:
-    """out/q: [B, Hq, D]; block_tables int32 [B, max_blocks]; context_lens int32 [B]."""
+              workspace: Optional[torch.Tensor] = None, stream=None, window: int = 0,
+              alibi_slopes: Optional[torch.Tensor] = None) -> None:
+    """out/q: [B, Hq, D]; block_tables int32 [B, max_blocks]; context_lens int32 [B].
+    window / alibi_slopes select pa_decode_ex's sliding window and ALiBi."""
     B, hq, d = q.shape
     lib = load_library()
     need = lib.pa_decode_workspace_size(B, hq, d, max_context_len, partition_size)
     workspace, wbytes = _workspace(need, q.device, workspace)
     desc = cache_desc(k_cache, k_scale, v_scale)
-    st = lib.pa_decode(_ptr(out), dtype_code(out.dtype), _ptr(q), dtype_code(q.dtype), B, hq,
-                       _ptr(k_cache), _ptr(v_cache), ctypes.byref(desc), _ptr(block_tables),
-                       block_tables.shape[1], _ptr(context_lens), int(max_context_len),
-                       float(scale), int(partition_size), _ptr(workspace), wbytes,
-                       _stream(stream))
-    _check(st, "pa_decode")
+    args = (_ptr(out), dtype_code(out.dtype), _ptr(q), dtype_code(q.dtype), B, hq,
+            _ptr(k_cache), _ptr(v_cache), ctypes.byref(desc), _ptr(block_tables),
+            block_tables.shape[1], _ptr(context_lens), int(max_context_len), float(scale),
+            int(partition_size))
+    opts = _options(window, alibi_slopes)
+    if opts is None:
+        st = lib.pa_decode(*args, _ptr(workspace), wbytes, _stream(stream))
+        _check(st, "pa_decode")
+    else:
+        st = lib.pa_decode_ex(*args, opts, _ptr(workspace), wbytes, _stream(stream))
+        _check(st, "pa_decode_ex")
 
 
 def pa_varlen(out: torch.Tensor, q: torch.Tensor, cu_seqlens_q: torch.Tensor,
               seqlens_k: torch.Tensor, max_q_len: int, max_context_len: int,
               k_cache: torch.Tensor, v_cache: torch.Tensor, block_tables: torch.Tensor,
               scale: float, k_scale=None, v_scale=None, workspace: Optional[torch.Tensor] = None,
-              stream=None) -> None:
-    """out/q: [total_q, Hq, D]; cu_seqlens_q int32 [S+1]; seqlens_k int32 [S]."""
+              stream=None, window: int = 0, alibi_slopes: Optional[torch.Tensor] = None) -> None:
+    """out/q: [total_q, Hq, D]; cu_seqlens_q int32 [S+1]; seqlens_k int32 [S].
+    window / alibi_slopes select pa_varlen_ex's sliding window and ALiBi."""
     total_q, hq, d = q.shape
     S = seqlens_k.shape[0]
     lib = load_library()
     need = lib.pa_varlen_workspace_size(S, total_q, hq, d, max_context_len)
     workspace, wbytes = _workspace(need, q.device, workspace)
     desc = cache_desc(k_cache, k_scale, v_scale)
-    st = lib.pa_varlen(_ptr(out), dtype_code(out.dtype), _ptr(q), dtype_code(q.dtype), total_q,
-                       S, hq, _ptr(cu_seqlens_q), _ptr(seqlens_k), int(max_q_len),
-                       int(max_context_len), _ptr(k_cache), _ptr(v_cache), ctypes.byref(desc),
-                       _ptr(block_tables), block_tables.shape[1], float(scale), _ptr(workspace),
-                       wbytes, _stream(stream))
-    _check(st, "pa_varlen")
+    args = (_ptr(out), dtype_code(out.dtype), _ptr(q), dtype_code(q.dtype), total_q, S, hq,
+            _ptr(cu_seqlens_q), _ptr(seqlens_k), int(max_q_len), int(max_context_len),
+            _ptr(k_cache), _ptr(v_cache), ctypes.byref(desc), _ptr(block_tables),
+            block_tables.shape[1], float(scale))
+    opts = _options(window, alibi_slopes)
+    if opts is None:
+        st = lib.pa_varlen(*args, _ptr(workspace), wbytes, _stream(stream))
+        _check(st, "pa_varlen")
+    else:
+        st = lib.pa_varlen_ex(*args, opts, _ptr(workspace), wbytes, _stream(stream))
+        _check(st, "pa_varlen_ex")
 
 
 def pa_device_error(stream=None) -> int:

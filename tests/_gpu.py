@@ -51,6 +51,8 @@ class DeviceStep:
             n = pa.pa_varlen_workspace_size(W.num_seqs, W.total_q, W.num_q_heads, W.head_dim,
                                             W.max_context_len)
         self.workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=dev)
+        self.window = 0            # sliding window / ALiBi for pa_decode_ex / pa_varlen_ex
+        self.alibi = None
 
     def fill_cache(self, chunk=1 << 18):
         """Write the cached context (outside any timed region), in pieces."""
@@ -79,11 +81,12 @@ class DeviceStep:
             pa.pa_decode(self.out, self.q, self.k_cache, self.v_cache, self.block_tables,
                          self.seqlens_k, W.max_context_len, W.scale, self.k_scale, self.v_scale,
                          W.partition_size if partition_size is None else partition_size,
-                         self.workspace)
+                         self.workspace, window=self.window, alibi_slopes=self.alibi)
         else:
             pa.pa_varlen(self.out, self.q, self.cu, self.seqlens_k, W.max_q_len,
                          W.max_context_len, self.k_cache, self.v_cache, self.block_tables,
-                         W.scale, self.k_scale, self.v_scale, self.workspace)
+                         W.scale, self.k_scale, self.v_scale, self.workspace,
+                         window=self.window, alibi_slopes=self.alibi)
 
     def step(self, **kw):
         self.write_new()
