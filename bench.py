@@ -70,7 +70,16 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def algorithmic_bytes(W) -> dict:
+def visible_keys(W, window: int) -> np.ndarray:
+    """Keys each request's attention must read: all of them, or with a
+    sliding window the last window + q_len - 1 (the span its rows see)."""
+    L = W.seqlens_k.astype(np.int64)
+    if window and window > 0:
+        return np.minimum(L, window + W.q_lens.astype(np.int64) - 1)
+    return L
+
+
+def algorithmic_bytes(W, window: int = 0) -> dict:
     """Bytes the step must move at least once from HBM: every distinct visible
     K/V slot of every KV head (a block shared by several sequences counts
     once; it is read from L2 after that), the queries, the outputs, the
@@ -78,6 +87,10 @@ def algorithmic_bytes(W) -> dict:
     'kv_logical' counts shared blocks once per sequence (the effective rate)."""
     kv_logical = W.kv_bytes_read()
     kv = W.unique_kv_bytes_read()
+    if window and window > 0:
+        per_tok = 2 * W.num_kv_heads * W.head_dim * W.kv_elem_bytes()
+        kv_logical = int(visible_keys(W, window).sum()) * per_tok
+        kv = min(kv, kv_logical)
     q = W.total_q * W.num_q_heads * W.head_dim * 2
     out = W.total_q * W.num_q_heads * W.head_dim * (4 if W.out_dtype == wl.F32 else 2)
     tbl = int((-(-W.seqlens_k.astype(np.int64) // W.block_size)).sum()) * 4 + W.num_seqs * 4
@@ -164,16 +177,20 @@ class ClockSampler:
 # --------------------------------------------------------------------------
 
 def dist_setup(n_gpus):
+    """One process per GPU (torchrun sets RANK / LOCAL_RANK / WORLD_SIZE): NCCL
+    for the timing reduction when CUDA is there, gloo otherwise (CPU tests)."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if world > 1:
-        import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return rank, world, local
@@ -186,11 +203,13 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The slowest replica's time: the job-level figure for weak scaling."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -341,7 +360,7 @@ def run_native(args):
             dist.destroy_process_group()
         return
 
-    by = algorithmic_bytes(W)
+    by = algorithmic_bytes(W, args.window)
     peak, peak_kind = peaks()
     gbs = by["kv"] * world / (ms * 1e-3) / 1e9
     attn_gbs = by["attention"] / (attn_ms * 1e-3) / 1e9

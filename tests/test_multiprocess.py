@@ -1,0 +1,44 @@
+"""The N-replica plumbing of bench.py on CPU: two gloo ranks, each timing its
+own replica, reduce to the slowest rank's time; only rank 0 reports."""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _rank(rank, world, port, q):
+    os.environ.update({"RANK": str(rank), "LOCAL_RANK": str(rank), "WORLD_SIZE": str(world),
+                       "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    import sys
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+    import torch.distributed as dist
+    r, w, _ = bench.dist_setup(world)
+    bench.barrier(w)
+    ms = bench.max_over_ranks(1.0 + r, w)            # rank r "took" 1 + r ms
+    q.put((r, w, ms, dist.get_backend()))
+    dist.destroy_process_group()
+
+
+def test_two_replicas_reduce_to_the_slowest():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    got = sorted(q.get(timeout=10) for _ in range(2))
+    assert [g[0] for g in got] == [0, 1]
+    assert all(g[1] == 2 and g[2] == 2.0 and g[3] == "gloo" for g in got)
