@@ -17,12 +17,14 @@
 //                    bf16/f16 hi + lo halves back into the same TMEM columns;
 //   O += P V         tcgen05.mma with A = P straight from TMEM and B = V from
 //                    shared memory (MN-major), D = O in TMEM.
-// Softmax is taken in two passes over the keys (pass 1: row max and sum; pass
-// 2: normalised P), so O never needs rescaling.  Warp roles: warps 0-3 own
-// the 128 rows (TMEM lanes), warp 4 issues the TMA loads (paged K/V tiles are
-// gathered block by block: 8 boxes of 16 tokens per 128-key tile), warp 5
-// allocates TMEM and issues the MMAs from one thread.  S/P live in two TMEM
-// buffers so the MMA of tile j+1 overlaps the softmax of tile j.
+// Softmax is online in one pass: P is taken against a running row maximum
+// that is only raised (and O, l rescaled in TMEM / registers) when a tile's
+// maximum exceeds it by more than 2^8, so P <= 256 and rescaling is rare.
+// Warp roles: 8 softmax warps (two per TMEM lane quarter, each owning 64 key
+// columns of S and 64 dimensions of O), 4 TMA producer warps (paged K/V
+// tiles are gathered 16 tokens at a time), 1 warp that allocates TMEM and
+// issues the MMAs from one thread.  S/P live in three TMEM buffers so the MMA
+// of tile j+1 overlaps the softmax of tile j.
 #include "pa_device.cuh"
 #include "pa_launch.h"
 
@@ -46,8 +48,9 @@ constexpr int kKOff = kQBytes;
 constexpr int kVOff = kKOff + kKStages * kTileBytes;
 constexpr int kTblMax = 2048;            // block-table entries cached in shared memory
 constexpr int kTblOff = kVOff + kVStages * kTileBytes;
-constexpr int kRedOff = kTblOff + kTblMax * 4;          // [2][128] floats, max then sum
-constexpr int kBarBase = kRedOff + 2 * 128 * 4;
+constexpr int kRedOff = kTblOff + kTblMax * 4;   // [2 slots][2 halves][128] maxima, [2][128] sums
+constexpr int kBarBase = kRedOff + 6 * 128 * 4;
+constexpr float kRescaleGap = 8.f;       // raise the running max when exceeded by 2^8
 // barriers: Q | K full x3 | K empty x3 | V full x2 | V empty x2 | S full x3 | P full x3 |
 //           PV done x3 | O
 enum { B_Q = 0, B_KF = 1, B_KE = 4, B_VF = 7, B_VE = 9, B_SF = 11, B_PF = 14, B_PVD = 17,
@@ -109,7 +112,7 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
   // are skipped (tiles jlo .. nkv-1 are visited, ntile of them)
   const int jlo = a.window > 0 ? max(0, pos0 - a.window + 1) / kBN : 0;
   const int ntile = nkv - jlo;
-  const int n_iter = 2 * ntile;
+  const int n_iter = ntile;
   const int hq0 = h * G;
 
   if (threadIdx.x == 0) {
@@ -167,7 +170,7 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
       const uint64_t pol = l2_policy_evict_last();
       constexpr int kShareBytes = 4 * 2 * 2048;        // 4 blocks x 2 halves per warp
       const int nstage = is_v ? kVStages : kKStages;
-      const int ntiles = is_v ? ntile : n_iter;         // V only in pass 2
+      const int ntiles = ntile;
       uint64_t* full = &bars[is_v ? B_VF : B_KF];
       uint64_t* empty = &bars[is_v ? B_VE : B_KE];
       const CUtensorMap* map = is_v ? &vmap : &kmap;
@@ -175,7 +178,7 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
       uint32_t ph_e[kKStages] = {0, 0, 0};
       int issued = 0;
       for (int u = 0; u < ntiles && !*abort_flag; ++u) {
-        const int j = jlo + (is_v ? u : (u >= ntile ? u - ntile : u));   // key tile
+        const int j = jlo + u;                              // key tile
         const int st = u % nstage;
         if (u >= nstage) {
           if (!wait_or_abort(&empty[st], ph_e[st], abort_flag)) break;
@@ -225,22 +228,15 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
       uint32_t ph_pf[kSBufs] = {0, 0, 0}, ph_pvd[kSBufs] = {0, 0, 0};
       bool ok = wait_or_abort(&bars[B_Q], 0, abort_flag);
       const uint32_t q_addr = smem_u32(sQ);
-      bool first_pv = true;
       int next_s = 0;
       for (int it = 0; ok && it < n_iter; ++it) {
         // keep S one tile ahead of PV: reusing the buffer of tile next_s - 3
         // then waits only for PV(it - 2), while PV(it - 1) stays queued
         while (ok && next_s < n_iter && next_s <= it + 1) {
           const int sb = next_s % kSBufs;
-          if (next_s >= kSBufs) {                 // buffer sb held tile next_s - kSBufs
-            const int prev = next_s - kSBufs;
-            if (prev < ntile) {                   // softmax finished reading S(prev)
-              if (!(ok = wait_or_abort(&bars[B_PF + sb], ph_pf[sb], abort_flag))) break;
-              ph_pf[sb] ^= 1;
-            } else {                              // PV(prev) finished reading P(prev)
-              if (!(ok = wait_or_abort(&bars[B_PVD + sb], ph_pvd[sb], abort_flag))) break;
-              ph_pvd[sb] ^= 1;
-            }
+          if (next_s >= kSBufs) {                 // PV(next_s - 3) finished reading P
+            if (!(ok = wait_or_abort(&bars[B_PVD + sb], ph_pvd[sb], abort_flag))) break;
+            ph_pvd[sb] ^= 1;
           }
           const int ks = next_s % kKStages;
           if (!(ok = wait_or_abort(&bars[B_KF + ks], ph_kf[ks], abort_flag))) break;
@@ -259,27 +255,24 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
           ++next_s;
         }
         if (!ok) break;
-        if (it >= ntile) {
-          // O += P V once the softmax warps have written P(it) and V has landed
-          const int b = it % kSBufs;
-          if (!(ok = wait_or_abort(&bars[B_PF + b], ph_pf[b], abort_flag))) break;
-          ph_pf[b] ^= 1;
-          const int vs = (it - ntile) % kVStages;
-          if (!(ok = wait_or_abort(&bars[B_VF + vs], ph_vf[vs], abort_flag))) break;
-          ph_vf[vs] ^= 1;
-          tc_fence_after();
-          const uint32_t v_addr = smem_u32(smem + kVOff + vs * kTileBytes);
-          const uint32_t p_base = tmem + static_cast<uint32_t>(b * 128);
+        // O += P V once the softmax warps have written P(it) (and rescaled O)
+        const int b = it % kSBufs;
+        if (!(ok = wait_or_abort(&bars[B_PF + b], ph_pf[b], abort_flag))) break;
+        ph_pf[b] ^= 1;
+        const int vs = it % kVStages;
+        if (!(ok = wait_or_abort(&bars[B_VF + vs], ph_vf[vs], abort_flag))) break;
+        ph_vf[vs] ^= 1;
+        tc_fence_after();
+        const uint32_t v_addr = smem_u32(smem + kVOff + vs * kTileBytes);
+        const uint32_t p_base = tmem + static_cast<uint32_t>(b * 128);
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t vd = smem_desc_sw128(v_addr + kk * 2048, kHalf, 1024);
-            tc_mma_ts(tmem + kOCol, p_base + kk * 8, vd, kIdescPV, first_pv ? 0u : 1u);
-            first_pv = false;
-            tc_mma_ts(tmem + kOCol, p_base + 64 + kk * 8, vd, kIdescPV, 1u);
-          }
-          tc_commit(&bars[B_VE + vs]);
-          tc_commit(&bars[B_PVD + b]);
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t vd = smem_desc_sw128(v_addr + kk * 2048, kHalf, 1024);
+          tc_mma_ts(tmem + kOCol, p_base + kk * 8, vd, kIdescPV, (it == 0 && kk == 0) ? 0u : 1u);
+          tc_mma_ts(tmem + kOCol, p_base + 64 + kk * 8, vd, kIdescPV, 1u);
         }
+        tc_commit(&bars[B_VE + vs]);
+        tc_commit(&bars[B_PVD + b]);
       }
       tc_commit(&bars[B_O]);                 // every MMA issued above is complete
       if (!ok) (void)wait_or_abort(&bars[B_O], 0, abort_flag);
@@ -305,53 +298,16 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
     auto tile_full = [&](int j) {
       return j * kBN + kBN - 1 <= pos0 && (a.window <= 0 || j * kBN >= last_pos - a.window + 1);
     };
-    // -------- pass 1: row maximum of the logits
-    float m_x = -INFINITY;
-    for (int it = 0; it < ntile; ++it) {
-      const int b = it % kSBufs;
-      if (!wait_or_abort(&bars[B_SF + b], ph_sf[b], abort_flag)) { ok = false; break; }
-      ph_sf[b] ^= 1;
-      tc_fence_after();
-      const int j = jlo + it;
-      uint32_t raw[64];
-      tmem_ld32(lane_base + b * 128 + half * 64, *reinterpret_cast<uint32_t (*)[32]>(raw));
-      tmem_ld32(lane_base + b * 128 + half * 64 + 32,
-                *reinterpret_cast<uint32_t (*)[32]>(raw + 32));
-      tmem_wait_ld();
-      const int key0 = j * kBN + half * 64;
-      const float b0 = slope * static_cast<float>(key0 - pos);
-      float mx = -INFINITY;
-      if (tile_full(j)) {
-#pragma unroll
-        for (int n2 = 0; n2 < 32; ++n2) {
-          const uint64_t x = ffma2(f2(__uint_as_float(raw[2 * n2]), __uint_as_float(raw[2 * n2 + 1])),
-                                   c2, f2(b0 + slope * (2 * n2), b0 + slope * (2 * n2 + 1)));
-          mx = fmax3(mx, f2lo(x), f2hi(x));
-        }
-      } else {
-        const int nlo = row_ok ? lo_row - key0 : 64, nhi = row_ok ? pos - key0 : -1;
-#pragma unroll
-        for (int n = 0; n < 64; ++n)
-          if (n >= nlo && n <= nhi)
-            mx = fmaxf(mx, fmaf(__uint_as_float(raw[n]), c, b0 + slope * n));
-      }
-      m_x = fmaxf(m_x, mx);
-      tc_fence_before();
-      mbar_arrive(&bars[B_PF + b]);
-    }
-    red[half * 128 + t] = m_x;
-    named_bar(1, kSoftmaxThreads);
-    const float m_all = fmaxf(red[t], red[128 + t]);
-    const float m = (m_all == -INFINITY) ? 0.f : m_all;
+    // -------- one pass: online softmax with a lazily raised row maximum
+    float m_used = -INFINITY;                  // log2-domain running maximum (both halves)
     uint64_t l2 = f2(0.f, 0.f);
-    // -------- pass 2: unnormalised P = 2^(x - m) (hi + lo) and its row sum
-    for (int it = ntile; ok && it < n_iter; ++it) {
+    for (int it = 0; ok && it < n_iter; ++it) {
       const int b = it % kSBufs;
       if (!wait_or_abort(&bars[B_SF + b], ph_sf[b], abort_flag)) { ok = false; break; }
       ph_sf[b] ^= 1;
       tc_fence_after();
-      const int vi = it - ntile;                 // position in the V ring sequence
-      const int j = jlo + vi;
+      const int vi = it;                         // position in the V ring sequence
+      const int j = jlo + it;
       uint32_t raw[64];
       tmem_ld32(lane_base + b * 128 + half * 64, *reinterpret_cast<uint32_t (*)[32]>(raw));
       tmem_ld32(lane_base + b * 128 + half * 64 + 32,
@@ -361,17 +317,62 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
       const bool full = tile_full(j);
       const int nlo = full ? 0 : (row_ok ? lo_row - key0 : 64);
       const int nhi = full ? 63 : (row_ok ? pos - key0 : -1);
-      const float b0 = slope * static_cast<float>(key0 - pos) - m;
-      uint32_t hi[32], lo[32];
+      const float b0 = slope * static_cast<float>(key0 - pos);
+      // logits x = s * scale * log2e + bias, in place; tile maximum over this half
+      float mx = -INFINITY;
 #pragma unroll
       for (int n2 = 0; n2 < 32; ++n2) {
         const uint64_t x = ffma2(f2(__uint_as_float(raw[2 * n2]), __uint_as_float(raw[2 * n2 + 1])),
                                  c2, f2(b0 + slope * (2 * n2), b0 + slope * (2 * n2 + 1)));
-        float p0 = fast_exp2(f2lo(x)), p1 = fast_exp2(f2hi(x));
+        float x0 = f2lo(x), x1 = f2hi(x);
         if (!full) {
-          p0 = (2 * n2 >= nlo && 2 * n2 <= nhi) ? p0 : 0.f;
-          p1 = (2 * n2 + 1 >= nlo && 2 * n2 + 1 <= nhi) ? p1 : 0.f;
+          x0 = (2 * n2 >= nlo && 2 * n2 <= nhi) ? x0 : -INFINITY;
+          x1 = (2 * n2 + 1 >= nlo && 2 * n2 + 1 <= nhi) ? x1 : -INFINITY;
         }
+        raw[2 * n2] = __float_as_uint(x0);
+        raw[2 * n2 + 1] = __float_as_uint(x1);
+        mx = fmax3(mx, x0, x1);
+      }
+      // row maximum of the tile: combine with the other half's columns
+      float* xch = red + (it & 1) * 256;
+      xch[half * 128 + t] = mx;
+      named_bar(3 + quarter, 64);
+      const float m_tile = fmaxf(xch[t], xch[128 + t]);
+      // raise the running maximum only when the tile exceeds it by 2^8
+      const bool raise = (m_used == -INFINITY) ? (m_tile != -INFINITY)
+                                               : (m_tile > m_used + kRescaleGap);
+      float alpha = 1.f;
+      if (raise) {
+        alpha = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - m_tile);
+        m_used = m_tile;
+      }
+      l2 = f2(f2lo(l2) * alpha, f2hi(l2) * alpha);
+      if (it > 0 && __any_sync(0xffffffffu, raise)) {
+        // O holds PV of earlier tiles: wait for PV(it - 1), then scale this
+        // warp's 64 dimensions of the rows that raised their maximum
+        const int pb = (it - 1) % kSBufs;
+        if (!wait_or_abort(&bars[B_PVD + pb], ((it - 1) / kSBufs) & 1, abort_flag)) {
+          ok = false;
+        }
+        tc_fence_after();
+#pragma unroll 1
+        for (int q2 = 0; q2 < 2; ++q2) {
+          uint32_t o[32];
+          tmem_ld32(lane_base + kOCol + half * 64 + 32 * q2, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(lane_base + kOCol + half * 64 + 32 * q2, o);
+        }
+      }
+      const float mu = (m_used == -INFINITY) ? 0.f : m_used;
+      const uint64_t nm2 = f2(-mu, -mu);
+      uint32_t hi[32], lo[32];
+#pragma unroll
+      for (int n2 = 0; n2 < 32; ++n2) {
+        const uint64_t x = fadd2(f2(__uint_as_float(raw[2 * n2]), __uint_as_float(raw[2 * n2 + 1])),
+                                 nm2);
+        const float p0 = fast_exp2(f2lo(x)), p1 = fast_exp2(f2hi(x));   // 2^-inf = 0
         const uint64_t p = f2(p0, p1);
         l2 = fadd2(l2, p);
         const uint32_t hw = pack2<BF16>(p0, p1);
@@ -405,9 +406,9 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
       mbar_arrive(&bars[B_PF + b]);
     }
     // -------- epilogue: O row / l -> out (this warp's 64 of the 128 dims)
-    red[half * 128 + t] = f2lo(l2) + f2hi(l2);
+    red[512 + half * 128 + t] = f2lo(l2) + f2hi(l2);
     named_bar(1, kSoftmaxThreads);
-    const float l_row = red[t] + red[128 + t];
+    const float l_row = red[512 + t] + red[512 + 128 + t];
     const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
     if (ok && wait_or_abort(&bars[B_O], 0, abort_flag)) {
       tc_fence_after();
