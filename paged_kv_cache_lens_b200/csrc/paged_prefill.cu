@@ -14,26 +14,29 @@
 //   S = Q K^T        tcgen05.mma kind::f16, A = Q and B = K from shared memory
 //                    (128-byte swizzle, K-major), D = S in TMEM (fp32);
 //   P = softmax row  one thread per row reads its TMEM lane, writes P as
-//                    bf16/f16 hi + lo halves back into the same TMEM columns;
+//                    bf16/f16 hi + lo halves back over the S columns it has read;
 //   O += P V         tcgen05.mma with A = P straight from TMEM and B = V from
 //                    shared memory (MN-major), D = O in TMEM.
 // Softmax is online in one pass: P is taken against a running row maximum
 // that is only raised (and O, l rescaled in TMEM / registers) when a tile's
 // maximum exceeds it by more than 2^8, so P <= 256 and rescaling is rare.
-// Warp roles: 8 softmax warps (two per TMEM lane quarter, each owning 64 key
-// columns of S and 64 dimensions of O), 4 TMA producer warps (paged K/V
-// tiles are gathered 16 tokens at a time), 1 warp that allocates TMEM and
-// issues the MMAs from one thread.  S/P live in three TMEM buffers so the MMA
-// of tile j+1 overlaps the softmax of tile j.
+// Warp roles: 8 softmax warps in two groups of four that take alternate key
+// tiles (one thread per tile row, all 128 columns); a group passes the row
+// maxima it used to the other through shared memory, so the exponentials of
+// one group overlap the TMEM loads, maxima and stores of the other.  4 TMA
+// producer warps (paged K/V tiles are gathered 16 tokens at a time), 1 warp
+// that allocates TMEM and issues the MMAs from one thread.  S/P live in three
+// TMEM buffers: S runs up to two tiles ahead of PV.
 #include "pa_device.cuh"
 #include "pa_launch.h"
 
 namespace pa {
 namespace {
 
-constexpr int kSoftmaxWarps = 8;         // two warps per TMEM lane quarter, 64 columns each
+constexpr int kSoftmaxWarps = 8;         // two groups of four: even and odd key tiles
 constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
-constexpr int kProducerWarps = 4;        // warps 0-1 of these stream K, 2-3 stream V
+constexpr int kGroupThreads = kSoftmaxThreads / 2;
+constexpr int kProducerWarps = 2;        // one streams K tiles, one V tiles
 constexpr int kProducerWarp0 = 8;
 constexpr int kMmaWarp = kProducerWarp0 + kProducerWarps;
 constexpr int kPfThreads = (kMmaWarp + 1) * 32;
@@ -48,13 +51,13 @@ constexpr int kKOff = kQBytes;
 constexpr int kVOff = kKOff + kKStages * kTileBytes;
 constexpr int kTblMax = 2048;            // block-table entries cached in shared memory
 constexpr int kTblOff = kVOff + kVStages * kTileBytes;
-constexpr int kRedOff = kTblOff + kTblMax * 4;   // [2 slots][2 halves][128] maxima, [2][128] sums
-constexpr int kBarBase = kRedOff + 6 * 128 * 4;
+constexpr int kRedOff = kTblOff + kTblMax * 4;   // [2 slots][128] maxima, [2 groups][128] sums
+constexpr int kBarBase = kRedOff + 4 * 128 * 4;
 constexpr float kRescaleGap = 8.f;       // raise the running max when exceeded by 2^8
 // barriers: Q | K full x3 | K empty x3 | V full x2 | V empty x2 | S full x3 | P full x3 |
-//           PV done x3 | O
+//           PV done x3 | O | row maxima published [2 slots][4 lane quarters]
 enum { B_Q = 0, B_KF = 1, B_KE = 4, B_VF = 7, B_VE = 9, B_SF = 11, B_PF = 14, B_PVD = 17,
-       B_O = 20, kNumBars = 21 };
+       B_O = 20, B_MX = 21, kNumBars = 29 };
 constexpr int kSmemBytes = kBarBase + kNumBars * 8 + 16 + 1024;
 constexpr uint32_t kTmemCols = 512;      // S/P buffers at columns 0, 128, 256; O at 384
 constexpr uint32_t kOCol = 384;
@@ -118,19 +121,20 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
   if (threadIdx.x == 0) {
     mbar_init(&bars[B_Q], 1);
     for (int s = 0; s < kKStages; ++s) {
-      mbar_init(&bars[B_KF + s], 2);
+      mbar_init(&bars[B_KF + s], 1);
       mbar_init(&bars[B_KE + s], 1);
     }
     for (int s = 0; s < kVStages; ++s) {
-      mbar_init(&bars[B_VF + s], 2);
+      mbar_init(&bars[B_VF + s], 1);
       mbar_init(&bars[B_VE + s], 1);
     }
     for (int s = 0; s < kSBufs; ++s) {
       mbar_init(&bars[B_SF + s], 1);
-      mbar_init(&bars[B_PF + s], kSoftmaxThreads);
+      mbar_init(&bars[B_PF + s], kGroupThreads);
       mbar_init(&bars[B_PVD + s], 1);
     }
     mbar_init(&bars[B_O], 1);
+    for (int s = 0; s < 8; ++s) mbar_init(&bars[B_MX + s], 32);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -145,255 +149,272 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
 
   if (warp >= kProducerWarp0 && warp < kMmaWarp) {
     // ================================================================ TMA producers
-    // Two warps stream K tiles (both passes) and two stream V tiles (pass 2),
-    // each loading 4 of the tile's 8 blocks (both 64-column halves) and
-    // arming its share of the expected bytes, so the K ring (3 deep) never
-    // waits behind V.
+    // One warp streams K tiles, one V tiles.  Lane 0 waits for a free stage
+    // and arms its barrier with the tile's bytes; lanes 0-7 then each fetch
+    // one 16-key sub-tile (both 64-column halves) through the block table.
     const int pw = warp - kProducerWarp0;
-    const bool is_v = pw >= 2;
-    const int sub = pw & 1;                           // blocks 4*sub .. 4*sub+3
+    const bool is_v = pw == 1;
     const int32_t* bt = a.block_tables + static_cast<int64_t>(r) * a.max_blocks_per_seq;
     const int bs = a.block_size;
     const int nblk = last_pos / bs + 1;               // blocks holding visible keys
     const int ncache = min(nblk, kTblMax);
     for (int i = pw * 32 + lane; i < ncache; i += kProducerWarps * 32) tbl[i] = __ldg(bt + i);
     named_bar(2, kProducerWarps * 32);
+    const int oob_row = a.num_blocks * a.num_kv_heads * bs;
+    if (pw == 0 && lane == 0) {
+      prefetch_tensormap(&kmap);
+      prefetch_tensormap(&vmap);
+      mbar_arrive_expect_tx(&bars[B_Q], kQBytes);
+      tma_load_3d(sQ, &qmap, 0, hq0, cu0 + qt * TQ, &bars[B_Q]);
+      tma_load_3d(sQ + kHalf, &qmap, 64, hq0, cu0 + qt * TQ, &bars[B_Q]);
+    }
+    const uint64_t pol = l2_policy_evict_last();
+    const int nstage = is_v ? kVStages : kKStages;
+    uint64_t* full = &bars[is_v ? B_VF : B_KF];
+    uint64_t* empty = &bars[is_v ? B_VE : B_KE];
+    const CUtensorMap* map = is_v ? &vmap : &kmap;
+    uint8_t* ring = smem + (is_v ? kVOff : kKOff);
+    int issued = 0;
+    for (int u = 0; u < ntile; ++u) {
+      const int j = jlo + u;                              // key tile
+      const int st = u % nstage;
+      int go = 1;
+      if (lane == 0) {
+        go = !*abort_flag;
+        if (go && u >= nstage) go = wait_or_abort(&empty[st], (u / nstage - 1) & 1, abort_flag);
+        if (go) mbar_arrive_expect_tx(&full[st], kTileBytes);
+      }
+      if (!__shfl_sync(0xffffffffu, go, 0)) break;
+      if (lane < 8) {
+        // sub-tile `lane` of key tile j: one box of 16 rows (two of 8 rows
+        // for 8-token blocks); past the visible keys the box starts past the
+        // pool and is zero filled
+        const int sti = j * 8 + lane;
+        int y0 = oob_row, y1 = bs == 8 ? oob_row : -1;
+        if (sti * 16 <= last_pos) {
+          const int32_t* src = (sti + 1) * 16 / bs + 1 < kTblMax ? tbl : bt;
+          int r0, r1;
+          if (tile_rows(src, sti, bs, nblk, a.num_blocks, a.num_kv_heads, h, oob_row, r0, r1)) {
+            y0 = r0;
+            y1 = r1;
+          } else {
+            report_error(kErrBlockRange);
+          }
+        }
+        uint8_t* box = ring + st * kTileBytes + lane * 2048;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          tma_load_2d(box + half * kHalf, map, half * 64, y0, &full[st], pol);
+          if (y1 >= 0) tma_load_2d(box + half * kHalf + 1024, map, half * 64, y1, &full[st], pol);
+        }
+      }
+      issued = u + 1;
+    }
+    // the last copies into each stage have landed before the CTA may exit
     if (lane == 0) {
-      const int oob_row = a.num_blocks * a.num_kv_heads * bs;
-      if (pw == 0) {
-        prefetch_tensormap(&kmap);
-        prefetch_tensormap(&vmap);
-        mbar_arrive_expect_tx(&bars[B_Q], kQBytes);
-        tma_load_3d(sQ, &qmap, 0, hq0, cu0 + qt * TQ, &bars[B_Q]);
-        tma_load_3d(sQ + kHalf, &qmap, 64, hq0, cu0 + qt * TQ, &bars[B_Q]);
-      }
-      const uint64_t pol = l2_policy_evict_last();
-      constexpr int kShareBytes = 4 * 2 * 2048;        // 4 blocks x 2 halves per warp
-      const int nstage = is_v ? kVStages : kKStages;
-      const int ntiles = ntile;
-      uint64_t* full = &bars[is_v ? B_VF : B_KF];
-      uint64_t* empty = &bars[is_v ? B_VE : B_KE];
-      const CUtensorMap* map = is_v ? &vmap : &kmap;
-      uint8_t* ring = smem + (is_v ? kVOff : kKOff);
-      uint32_t ph_e[kKStages] = {0, 0, 0};
-      int issued = 0;
-      for (int u = 0; u < ntiles && !*abort_flag; ++u) {
-        const int j = jlo + u;                              // key tile
-        const int st = u % nstage;
-        if (u >= nstage) {
-          if (!wait_or_abort(&empty[st], ph_e[st], abort_flag)) break;
-          ph_e[st] ^= 1;
-        }
-        // this warp's four 16-key sub-tiles of key tile j (one box of 16 rows,
-        // or two of 8 rows for 8-token blocks); past the visible keys the box
-        // starts past the pool and is zero filled
-        int ys[4], ys1[4];
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const int sti = j * 8 + 4 * sub + b;
-          ys[b] = oob_row;
-          ys1[b] = bs == 8 ? oob_row : -1;
-          if (sti * 16 <= last_pos) {
-            const int32_t* src = (sti + 1) * 16 / bs + 1 < kTblMax ? tbl : bt;
-            int y0, y1;
-            if (tile_rows(src, sti, bs, nblk, a.num_blocks, a.num_kv_heads, h, oob_row, y0, y1)) {
-              ys[b] = y0;
-              ys1[b] = y1;
-            } else {
-              report_error(kErrBlockRange);
-            }
-          }
-        }
-        uint8_t* dst = ring + st * kTileBytes;
-        mbar_arrive_expect_tx(&full[st], kShareBytes);
-#pragma unroll
-        for (int b = 0; b < 4; ++b)
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            uint8_t* box = dst + half * kHalf + (4 * sub + b) * 2048;
-            tma_load_2d(box, map, half * 64, ys[b], &full[st], pol);
-            if (ys1[b] >= 0) tma_load_2d(box + 1024, map, half * 64, ys1[b], &full[st], pol);
-          }
-        issued = u + 1;
-      }
-      // the last copies into each stage have landed before the CTA may exit
       for (int u = issued - 1; u >= 0 && u >= issued - nstage; --u)
         (void)mbar_wait_bounded(&full[u % nstage], (u / nstage) & 1);
       if (pw == 0) (void)mbar_wait_bounded(&bars[B_Q], 0);
     }
   } else if (warp == kMmaWarp) {
     // ================================================================ MMA issuer
-    if (lane == 0) {
-      uint32_t ph_kf[kKStages] = {0, 0, 0}, ph_vf[kVStages] = {0, 0};
-      uint32_t ph_pf[kSBufs] = {0, 0, 0}, ph_pvd[kSBufs] = {0, 0, 0};
-      bool ok = wait_or_abort(&bars[B_Q], 0, abort_flag);
-      const uint32_t q_addr = smem_u32(sQ);
-      int next_s = 0;
-      for (int it = 0; ok && it < n_iter; ++it) {
-        // keep S one tile ahead of PV: reusing the buffer of tile next_s - 3
-        // then waits only for PV(it - 2), while PV(it - 1) stays queued
-        while (ok && next_s < n_iter && next_s <= it + 1) {
-          const int sb = next_s % kSBufs;
-          if (next_s >= kSBufs) {                 // PV(next_s - 3) finished reading P
-            if (!(ok = wait_or_abort(&bars[B_PVD + sb], ph_pvd[sb], abort_flag))) break;
-            ph_pvd[sb] ^= 1;
-          }
-          const int ks = next_s % kKStages;
-          if (!(ok = wait_or_abort(&bars[B_KF + ks], ph_kf[ks], abort_flag))) break;
-          ph_kf[ks] ^= 1;
-          tc_fence_after();
-          const uint32_t k_addr = smem_u32(smem + kKOff + ks * kTileBytes);
-          const uint32_t d = tmem + static_cast<uint32_t>(sb * 128);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;
-            tc_mma_ss(d, smem_desc_sw128(q_addr + off, 16, 1024),
-                      smem_desc_sw128(k_addr + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
-          }
-          tc_commit(&bars[B_SF + sb]);
-          tc_commit(&bars[B_KE + ks]);            // S is the only reader of K
-          ++next_s;
-        }
-        if (!ok) break;
-        // O += P V once the softmax warps have written P(it) (and rescaled O)
-        const int b = it % kSBufs;
-        if (!(ok = wait_or_abort(&bars[B_PF + b], ph_pf[b], abort_flag))) break;
-        ph_pf[b] ^= 1;
-        const int vs = it % kVStages;
-        if (!(ok = wait_or_abort(&bars[B_VF + vs], ph_vf[vs], abort_flag))) break;
-        ph_vf[vs] ^= 1;
+    // The whole warp runs this loop converged (every wait is taken by all
+    // lanes, and agreed on); one elected lane issues each MMA and commit.
+    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, wait_or_abort(bar, parity, abort_flag));
+    };
+    bool ok = wait_all(&bars[B_Q], 0);
+    // descriptors of the first 16-column slice of Q, K stage 0 and V stage 0;
+    // a slice or stage is an offset added to the start-address field (byte
+    // address / 16, which stays below 2^14 for any shared-memory address)
+    const uint64_t q_desc = smem_desc_sw128(smem_u32(sQ), 16, 1024);
+    const uint64_t k_desc = smem_desc_sw128(smem_u32(smem + kKOff), 16, 1024);
+    const uint64_t v_desc = smem_desc_sw128(smem_u32(smem + kVOff), kHalf, 1024);
+    int next_s = 0;
+    for (int it = 0; ok && it < n_iter; ++it) {
+      // S runs up to two tiles ahead of PV, so both softmax groups have a
+      // tile to work on; buffer reuse waits for PV(next_s - 3) only
+      while (ok && next_s < n_iter && next_s <= it + 2) {
+        const int sb = next_s % kSBufs;
+        if (next_s >= kSBufs && !(ok = wait_all(&bars[B_PVD + sb], (next_s / kSBufs - 1) & 1)))
+          break;
+        const int ks = next_s % kKStages;
+        if (!(ok = wait_all(&bars[B_KF + ks], (next_s / kKStages) & 1))) break;
         tc_fence_after();
-        const uint32_t v_addr = smem_u32(smem + kVOff + vs * kTileBytes);
-        const uint32_t p_base = tmem + static_cast<uint32_t>(b * 128);
+        const uint64_t kd = k_desc + static_cast<uint64_t>((ks * kTileBytes) >> 4);
+        const uint32_t d = tmem + static_cast<uint32_t>(sb * 128);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t vd = smem_desc_sw128(v_addr + kk * 2048, kHalf, 1024);
-          tc_mma_ts(tmem + kOCol, p_base + kk * 8, vd, kIdescPV, (it == 0 && kk == 0) ? 0u : 1u);
-          tc_mma_ts(tmem + kOCol, p_base + 64 + kk * 8, vd, kIdescPV, 1u);
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kHalf + (kk & 3) * 32) >> 4);
+          tc_mma_ss_warp(d, q_desc + off, kd + off, kIdescS, kk > 0 ? 1u : 0u);
         }
-        tc_commit(&bars[B_VE + vs]);
-        tc_commit(&bars[B_PVD + b]);
+        tc_commit_warp(&bars[B_SF + sb]);
+        tc_commit_warp(&bars[B_KE + ks]);       // S is the only reader of K
+        ++next_s;
       }
-      tc_commit(&bars[B_O]);                 // every MMA issued above is complete
-      if (!ok) (void)wait_or_abort(&bars[B_O], 0, abort_flag);
+      if (!ok) break;
+      // O += P V once the softmax group has written P(it) (and rescaled O)
+      const int b = it % kSBufs;
+      if (!(ok = wait_all(&bars[B_PF + b], (it / kSBufs) & 1))) break;
+      const int vs = it % kVStages;
+      if (!(ok = wait_all(&bars[B_VF + vs], (it / kVStages) & 1))) break;
+      tc_fence_after();
+      const uint64_t vd = v_desc + static_cast<uint64_t>((vs * kTileBytes) >> 4);
+      const uint32_t p_base = tmem + static_cast<uint32_t>(b * 128);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        // keys 16kk .. 16kk+15: chunk kk/2 of 32 keys holds 16 hi columns
+        // then 16 lo columns, 8 columns (16 packed values) per half chunk
+        const uint32_t pc = p_base + 32 * (kk >> 1) + 8 * (kk & 1);
+        const uint64_t vk = vd + static_cast<uint64_t>((kk * 2048) >> 4);
+        tc_mma_ts_warp(tmem + kOCol, pc, vk, kIdescPV, (it == 0 && kk == 0) ? 0u : 1u);
+        tc_mma_ts_warp(tmem + kOCol, pc + 16, vk, kIdescPV, 1u);
+      }
+      tc_commit_warp(&bars[B_VE + vs]);
+      tc_commit_warp(&bars[B_PVD + b]);
     }
+    tc_commit_warp(&bars[B_O]);              // every MMA issued above is complete
+    if (!ok) (void)wait_all(&bars[B_O], 0);
   } else {
     // ================================================================ softmax / epilogue
-    // Warp w owns TMEM lanes 32*(w%4).. (tile rows) and key columns 64*(w/4)..
-    const int quarter = warp & 3, half = warp >> 2;
+    // Group grp (warps 4*grp ..) takes key tiles grp, grp + 2, ...; warp w's
+    // 32 threads own tile rows (= TMEM lanes) 32*(w%4).., all 128 columns.
+    const int quarter = warp & 3, grp = warp >> 2;
     const int t = quarter * 32 + lane;         // tile row == TMEM lane
     const int i = t / G, g = t % G;
     const bool row_ok = i < rows_valid;
     const int pos = pos0 + i;
     const float c = a.scale * kLog2eF;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    uint32_t ph_sf[kSBufs] = {0, 0, 0};
     bool ok = true;
     // Row visibility: keys lo_row .. pos (lo_row from the sliding window);
     // logits in the log2 domain x = s*scale*log2e + slope*log2e*(key - pos).
     const int lo_row = a.window > 0 ? pos - a.window + 1 : 0;
     const float slope = a.alibi ? a.alibi[hq0 + g] * kLog2eF : 0.f;
-    const uint64_t c2 = f2(c, c);
+    // without ALiBi (and with scale > 0) the max is taken on the raw scores
+    // and the scale folds into the exponent's FFMA
+    const bool direct = a.alibi == nullptr && c > 0.f;
+    const float cc = direct ? c : 1.f;
     // a tile every row sees in full needs no mask
     auto tile_full = [&](int j) {
       return j * kBN + kBN - 1 <= pos0 && (a.window <= 0 || j * kBN >= last_pos - a.window + 1);
     };
-    // -------- one pass: online softmax with a lazily raised row maximum
-    float m_used = -INFINITY;                  // log2-domain running maximum (both halves)
-    uint64_t l2 = f2(0.f, 0.f);
-    for (int it = 0; ok && it < n_iter; ++it) {
-      const int b = it % kSBufs;
-      if (!wait_or_abort(&bars[B_SF + b], ph_sf[b], abort_flag)) { ok = false; break; }
-      ph_sf[b] ^= 1;
-      tc_fence_after();
-      const int vi = it;                         // position in the V ring sequence
-      const int j = jlo + it;
-      uint32_t raw[64];
-      tmem_ld32(lane_base + b * 128 + half * 64, *reinterpret_cast<uint32_t (*)[32]>(raw));
-      tmem_ld32(lane_base + b * 128 + half * 64 + 32,
-                *reinterpret_cast<uint32_t (*)[32]>(raw + 32));
-      tmem_wait_ld();
-      const int key0 = j * kBN + half * 64;
-      const bool full = tile_full(j);
-      const int nlo = full ? 0 : (row_ok ? lo_row - key0 : 64);
-      const int nhi = full ? 63 : (row_ok ? pos - key0 : -1);
-      const float b0 = slope * static_cast<float>(key0 - pos);
-      // logits x = s * scale * log2e + bias, in place; tile maximum over this half
-      float mx = -INFINITY;
+    // 32 columns of S (column0 = k0 .. k0 + 31 of the tile) -> logits in place
+    auto logits = [&](uint32_t (&v)[32], int col0, int nlo, int nhi, bool full, float b0) {
+      if (!direct) {
 #pragma unroll
-      for (int n2 = 0; n2 < 32; ++n2) {
-        const uint64_t x = ffma2(f2(__uint_as_float(raw[2 * n2]), __uint_as_float(raw[2 * n2 + 1])),
-                                 c2, f2(b0 + slope * (2 * n2), b0 + slope * (2 * n2 + 1)));
-        float x0 = f2lo(x), x1 = f2hi(x);
-        if (!full) {
-          x0 = (2 * n2 >= nlo && 2 * n2 <= nhi) ? x0 : -INFINITY;
-          x1 = (2 * n2 + 1 >= nlo && 2 * n2 + 1 <= nhi) ? x1 : -INFINITY;
+        for (int n = 0; n < 32; ++n)
+          v[n] = __float_as_uint(
+              fmaf(__uint_as_float(v[n]), c, fmaf(slope, static_cast<float>(col0 + n), b0)));
+      }
+      if (!full) {
+#pragma unroll
+        for (int n = 0; n < 32; ++n)
+          if (col0 + n < nlo || col0 + n > nhi) v[n] = __float_as_uint(-INFINITY);
+      }
+    };
+    float* m_pub = red;                        // [slot = tile & 1][row]: maximum used
+    float l_part = 0.f;                        // this group's share of the row sum,
+    float m_l = -INFINITY;                     // relative to 2^m_l
+    for (int it = grp; ok && it < n_iter; it += 2) {
+      const int b = it % kSBufs;
+      if (!wait_or_abort(&bars[B_SF + b], (it / kSBufs) & 1, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      const int j = jlo + it;
+      const int key0 = j * kBN;
+      const bool full = tile_full(j);
+      // keys outside lo_row .. pos of this row (every key of a padding row)
+      // are masked; stale slots past kv_len always fall in a masked tile
+      const int nlo = full ? 0 : (row_ok ? lo_row - key0 : kBN);
+      const int nhi = full ? kBN - 1 : (row_ok ? pos - key0 : -1);
+      const float b0 = slope * static_cast<float>(key0 - pos);
+      const uint32_t s_col = lane_base + b * 128;
+      // ---- the row of S (128 columns) in registers, one TMEM round trip;
+      // the tile's row maximum (log2 domain) in four independent chains
+      uint32_t v[4][32];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) tmem_ld32(s_col + 32 * k, v[k]);
+      tmem_wait_ld();
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        logits(v[k], 32 * k, nlo, nhi, full, b0);
+#pragma unroll
+        for (int n2 = 0; n2 < 16; ++n2)
+          m4[n2 & 3] = fmax3(m4[n2 & 3], __uint_as_float(v[k][2 * n2]), __uint_as_float(v[k][2 * n2 + 1]));
+      }
+      float m_tile = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      if (direct) m_tile *= c;                 // scale > 0: the maximum commutes with it
+      // ---- the running maximum before this tile, from the group that ran
+      // tile it - 1; raise it only when this tile exceeds it by 2^8
+      float m_prev = -INFINITY;
+      if (it > 0) {
+        const int sp = (it - 1) & 1;
+        if (!wait_or_abort(&bars[B_MX + 4 * sp + quarter], ((it - 1) >> 1) & 1, abort_flag)) {
+          ok = false;
+          break;
         }
-        raw[2 * n2] = __float_as_uint(x0);
-        raw[2 * n2 + 1] = __float_as_uint(x1);
-        mx = fmax3(mx, x0, x1);
+        m_prev = m_pub[sp * 128 + t];
       }
-      // row maximum of the tile: combine with the other half's columns
-      float* xch = red + (it & 1) * 256;
-      xch[half * 128 + t] = mx;
-      named_bar(3 + quarter, 64);
-      const float m_tile = fmaxf(xch[t], xch[128 + t]);
-      // raise the running maximum only when the tile exceeds it by 2^8
-      const bool raise = (m_used == -INFINITY) ? (m_tile != -INFINITY)
-                                               : (m_tile > m_used + kRescaleGap);
-      float alpha = 1.f;
-      if (raise) {
-        alpha = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - m_tile);
-        m_used = m_tile;
+      const bool raise = (m_prev == -INFINITY) ? (m_tile != -INFINITY)
+                                               : (m_tile > m_prev + kRescaleGap);
+      const float m_new = raise ? m_tile : m_prev;
+      m_pub[(it & 1) * 128 + t] = m_new;
+      mbar_arrive(&bars[B_MX + 4 * (it & 1) + quarter]);
+      if (m_new != m_l) {                      // rescale this group's partial sum
+        l_part = (m_l == -INFINITY) ? 0.f : l_part * fast_exp2(m_l - m_new);
+        m_l = m_new;
       }
-      l2 = f2(f2lo(l2) * alpha, f2hi(l2) * alpha);
+      // ---- p = 2^(x - m_new) per 32-column chunk, written back over the
+      // chunk's S columns as 16 hi then 16 lo columns of packed pairs
+      const float nmu = (m_new == -INFINITY) ? 0.f : -m_new;
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        uint32_t hi[16], lo[16];
+#pragma unroll
+        for (int n2 = 0; n2 < 16; ++n2) {
+          const float p0 = fast_exp2(fmaf(__uint_as_float(v[k][2 * n2]), cc, nmu));   // 2^-inf = 0
+          const float p1 = fast_exp2(fmaf(__uint_as_float(v[k][2 * n2 + 1]), cc, nmu));
+          ls[n2 & 3] += p0 + p1;
+          const uint32_t hw = pack2<BF16>(p0, p1);
+          hi[n2] = hw;
+          lo[n2] = pack2<BF16>(p0 - lo_half_to_float<BF16>(hw), p1 - lo_half_to_float<BF16>(hw >> 16));
+        }
+        tmem_st16(s_col + 32 * k, hi);
+        tmem_st16(s_col + 32 * k + 16, lo);
+      }
+      l_part += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       if (it > 0 && __any_sync(0xffffffffu, raise)) {
-        // O holds PV of earlier tiles: wait for PV(it - 1), then scale this
-        // warp's 64 dimensions of the rows that raised their maximum
-        const int pb = (it - 1) % kSBufs;
-        if (!wait_or_abort(&bars[B_PVD + pb], ((it - 1) / kSBufs) & 1, abort_flag)) {
+        // O holds PV of tiles < it: wait for PV(it - 1), then scale the rows
+        // that raised their maximum (alpha = 1 elsewhere, 0 for a row whose
+        // earlier keys were all masked)
+        const float alpha = !raise ? 1.f : (m_prev == -INFINITY ? 0.f : fast_exp2(m_prev - m_new));
+        if (!wait_or_abort(&bars[B_PVD + (it - 1) % kSBufs], ((it - 1) / kSBufs) & 1,
+                           abort_flag)) {
           ok = false;
         }
         tc_fence_after();
 #pragma unroll 1
-        for (int q2 = 0; q2 < 2; ++q2) {
+        for (int q2 = 0; q2 < 4; ++q2) {
           uint32_t o[32];
-          tmem_ld32(lane_base + kOCol + half * 64 + 32 * q2, o);
+          tmem_ld32(lane_base + kOCol + 32 * q2, o);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(lane_base + kOCol + half * 64 + 32 * q2, o);
+          tmem_st32(lane_base + kOCol + 32 * q2, o);
         }
       }
-      const float mu = (m_used == -INFINITY) ? 0.f : m_used;
-      const uint64_t nm2 = f2(-mu, -mu);
-      uint32_t hi[32], lo[32];
-#pragma unroll
-      for (int n2 = 0; n2 < 32; ++n2) {
-        const uint64_t x = fadd2(f2(__uint_as_float(raw[2 * n2]), __uint_as_float(raw[2 * n2 + 1])),
-                                 nm2);
-        const float p0 = fast_exp2(f2lo(x)), p1 = fast_exp2(f2hi(x));   // 2^-inf = 0
-        const uint64_t p = f2(p0, p1);
-        l2 = fadd2(l2, p);
-        const uint32_t hw = pack2<BF16>(p0, p1);
-        hi[n2] = hw;
-        const uint64_t r2 = fsub2(p, f2(lo_half_to_float<BF16>(hw), lo_half_to_float<BF16>(hw >> 16)));
-        lo[n2] = pack2<BF16>(f2lo(r2), f2hi(r2));
-      }
-      tmem_st32(lane_base + b * 128 + half * 32, hi);
-      tmem_st32(lane_base + b * 128 + 64 + half * 32, lo);
       // Keys of the context's partial last block that lie past kv_len hold
       // whatever the slot held; P is 0 there but 0 * NaN is NaN: clear them.
-      const int tile0 = j * kBN;
-      const int stale0 = kv_len, stale1 = min((kv_len + 15) & ~15, tile0 + kBN);
-      if (stale0 < stale1 && stale0 >= tile0) {
-        const int vs = vi % kVStages;
-        if (wait_or_abort(&bars[B_VF + vs], (vi / kVStages) & 1, abort_flag)) {
+      const int stale0 = kv_len, stale1 = min((kv_len + 15) & ~15, key0 + kBN);
+      if (stale0 < stale1 && stale0 >= key0) {
+        const int vs = it % kVStages;
+        if (wait_or_abort(&bars[B_VF + vs], (it / kVStages) & 1, abort_flag)) {
           uint8_t* sV = smem + kVOff + vs * kTileBytes;
           const int nrows = stale1 - stale0;
-          const int ts = threadIdx.x;
-          for (int idx = ts; idx < nrows * 16; idx += kSoftmaxThreads) {
-            const int row = stale0 - tile0 + idx / 16;
+          for (int idx = t; idx < nrows * 16; idx += kGroupThreads) {
+            const int row = stale0 - key0 + idx / 16;
             const int c16 = idx % 16;
             *reinterpret_cast<uint4*>(sV + (c16 >> 3) * kHalf + row * 128 + (c16 & 7) * 16) =
                 make_uint4(0, 0, 0, 0);
@@ -405,11 +426,15 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
       tc_fence_before();
       mbar_arrive(&bars[B_PF + b]);
     }
-    // -------- epilogue: O row / l -> out (this warp's 64 of the 128 dims)
-    red[512 + half * 128 + t] = f2lo(l2) + f2hi(l2);
+    // -------- epilogue: O row / l -> out (group grp writes dims 64*grp ..)
+    named_bar(1, kSoftmaxThreads);             // every tile's maximum is published
+    const float m_fin = n_iter > 0 ? m_pub[((n_iter - 1) & 1) * 128 + t] : -INFINITY;
+    red[256 + grp * 128 + t] =
+        (m_l == -INFINITY || m_fin == -INFINITY) ? 0.f : l_part * fast_exp2(m_l - m_fin);
     named_bar(1, kSoftmaxThreads);
-    const float l_row = red[512 + t] + red[512 + 128 + t];
+    const float l_row = red[256 + t] + red[384 + t];
     const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
+    const int half = grp;
     if (ok && wait_or_abort(&bars[B_O], 0, abort_flag)) {
       tc_fence_after();
       uint32_t o[64];
