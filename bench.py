@@ -70,6 +70,40 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+NOMINAL_HBM_GBS = 8000.0     # B200 HBM3e, nominal (context beside the measured copy peak)
+
+
+def read_probe_gbs(torch, pa, dev, stream, nbytes=2 << 30, iters=10) -> float:
+    """Read-only HBM ceiling on this GPU: the library's read probe streaming a
+    2 GiB buffer (16x the L2), CUDA events around `iters` launches."""
+    buf = torch.ones(nbytes // 4, dtype=torch.int32, device=dev)
+    sink = torch.zeros(1, dtype=torch.int32, device=dev)
+    for _ in range(3):
+        pa.pa_hbm_read_probe(buf, sink, stream)
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(iters):
+        pa.pa_hbm_read_probe(buf, sink, stream)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    gbs = nbytes * iters / (a.elapsed_time(b) * 1e-3) / 1e9
+    del buf
+    return gbs
+
+
+def chunk_flops(W, window: int, requests) -> int:
+    """Algorithmic FLOPs of the given requests' attention: 4*D per visible
+    (query row, query head, key) triple (QK^T and PV)."""
+    total = 0
+    for r in requests:
+        ql, L = int(W.q_lens[r]), int(W.seqlens_k[r])
+        pos = L - ql + np.arange(ql, dtype=np.int64)
+        vis = pos + 1 if not window or window <= 0 else np.minimum(pos + 1, window)
+        total += int(vis.sum())
+    return total * W.num_q_heads * 4 * W.head_dim
+
+
 def visible_keys(W, window: int) -> np.ndarray:
     """Keys each request's attention must read: all of them, or with a
     sliding window the last window + q_len - 1 (the span its rows see)."""
@@ -360,6 +394,14 @@ def run_native(args):
             dist.destroy_process_group()
         return
 
+    # ---- context measured after the timed region: read-only HBM ceiling and,
+    # for a mixed step, its decode rows and prefill chunks timed apart
+    probe = read_probe_gbs(torch, pa, dev, stream)
+    split = None
+    if not W.decode:
+        split = mixed_split(torch, pa, W, args, dev, stream, q, bt, sk, out, kc, vc, ks, vs,
+                            slopes)
+
     by = algorithmic_bytes(W, args.window)
     peak, peak_kind = peaks()
     gbs = by["kv"] * world / (ms * 1e-3) / 1e9
@@ -381,6 +423,7 @@ def run_native(args):
         "data": "synthetic (seeded N(0,1) q/K/V, seeded block tables)",
         "seq_steps_per_s_per_layer": round(seq_steps, 1),
         "pct_of_hbm_peak": round(100 * gbs / peak, 2),
+        "pct_of_nominal_hbm": round(100 * gbs / NOMINAL_HBM_GBS, 2),
         "config": {
             "workload": workload_name(W),
             "batch": W.num_seqs, "total_q": W.total_q, "q_heads": W.num_q_heads,
@@ -399,10 +442,16 @@ def run_native(args):
             "frac": round(attn_gbs / peak, 4), "traffic": traffic,
             "peak_source": f"{peak_kind} hbm_gbs", "attention_ms": round(attn_ms, 5),
             "algorithmic_bytes": by["attention"],
+            "nominal_peak": NOMINAL_HBM_GBS,
+            "frac_of_nominal": round(attn_gbs / NOMINAL_HBM_GBS, 4),
+            "read_probe_gbs": round(probe, 1),
+            "frac_of_read_probe": round(attn_gbs / probe, 4),
         },
         "clocks": clocks.summary(),
         "gpu_launches": launches_per_step * args.steps,
     }
+    if split:
+        line["split"] = split
     if e2e:
         e2e_ms, h2d, d2h = e2e
         line["e2e"] = {"value": round(by["kv"] * world / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
@@ -476,6 +525,57 @@ def _oracle_sample(W, n_seqs, threads):
     return dt_s, int(W.seqlens_k[:reqs].astype(np.int64).sum()) * per_tok, reqs
 
 
+def mixed_split(torch, pa, W, args, dev, stream, q, bt, sk, out, kc, vc, ks, vs, slopes,
+                iters=50):
+    """A mixed step whose leading requests are single-row decodes and the rest
+    prefill chunks: each part through pa_varlen on its own (same pools, same
+    rows), CUDA events over `iters` calls.  Decode rows report KV GB/s, chunks
+    algorithmic TFLOP/s."""
+    ql = W.q_lens
+    nd = 0
+    while nd < W.num_seqs and ql[nd] == 1:
+        nd += 1
+    if nd == 0 or nd == W.num_seqs or (ql[nd:] < 2).any():
+        return None
+    per_tok = 2 * W.num_kv_heads * W.head_dim * W.kv_elem_bytes()
+    vis = visible_keys(W, args.window)
+    res = {}
+    for name, r0, r1 in (("decode_rows", 0, nd), ("chunks", nd, W.num_seqs)):
+        q0, q1 = int(W.cu_seqlens_q[r0]), int(W.cu_seqlens_q[r1])
+        cu_s = torch.from_numpy((W.cu_seqlens_q[r0:r1 + 1] - W.cu_seqlens_q[r0])
+                                .astype(np.int32)).to(dev)
+        nws = pa.pa_varlen_workspace_size(r1 - r0, q1 - q0, W.num_q_heads, W.head_dim,
+                                          W.max_context_len)
+        ws_s = torch.empty(max(nws, 256), dtype=torch.uint8, device=dev)
+        mq = int(ql[r0:r1].max())
+
+        def call():
+            pa.pa_varlen(out[q0:q1], q[q0:q1], cu_s, sk[r0:r1], mq, W.max_context_len, kc, vc,
+                         bt[r0:r1], W.scale, ks, vs, ws_s, stream, window=args.window,
+                         alibi_slopes=slopes)
+
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(iters):
+            call()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = a.elapsed_time(b) / iters
+        part = {"requests": r1 - r0, "rows": q1 - q0, "ms": round(ms, 5)}
+        if name == "decode_rows":
+            kv = int(vis[r0:r1].sum()) * per_tok
+            part.update(kv_bytes=kv, kv_gbs=round(kv / (ms * 1e-3) / 1e9, 1))
+        else:
+            fl = chunk_flops(W, args.window, range(r0, r1))
+            part.update(algorithmic_flops=fl, tflops=round(fl / (ms * 1e-3) / 1e12, 1))
+        res[name] = part
+    assert pa.pa_device_error(stream) == 0
+    return res
+
+
 def cpu_baseline(W, budget_s=12.0):
     """The oracle, as it stands, on this host's cores: a sample of the step
     (first n requests) grown towards budget_s, then repeated until the budget
@@ -489,7 +589,14 @@ def cpu_baseline(W, budget_s=12.0):
     while total_t < budget_s:
         t, b, reqs = _oracle_sample(W, reqs, threads)
         total_t, total_b, reps = total_t + t, total_b + b, reps + 1
+    # one core, on the first request alone, for ~2 s
+    t1, b1, reps1 = 0.0, 0, 0
+    while t1 < 2.0:
+        t, b, _ = _oracle_sample(W, 1, 1)
+        t1, b1, reps1 = t1 + t, b1 + b, reps1 + 1
     return {"value": round(total_b / total_t / 1e9, 4), "unit": "GB/s", "cores": threads,
+            "single_core_value": round(b1 / t1 / 1e9, 4),
+            "single_core_sample": f"request 0 x {reps1} repeats, {t1:.1f} s",
             "kind": "oracle",
             "sample": f"{reqs} of {W.num_seqs} requests of the step (cache write + attention, "
                       f"fp64) x {reps} repeats, {total_t:.1f} s",

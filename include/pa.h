@@ -290,6 +290,20 @@ pa_status pa_varlen_ex(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_
                        void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Measurement helper, not part of the method (the pages have no counterpart):
+ * stream `bytes` of device memory at `buf` once with read-only 16-byte loads,
+ * the read-only bandwidth ceiling that the attention kernels' achieved GB/s
+ * is reported beside (the roofline denominator itself is a measured copy).
+ *
+ * buf    : device memory, 16-byte aligned; bytes a multiple of 16 (0 allowed).
+ * sink   : device uint32, 4-byte aligned; receives the XOR of all 32-bit
+ *          words of the buffer (exact; a check that every byte was read).
+ * Errors : PA_ERR_INVALID_ARG for misaligned or negative arguments,
+ *          PA_ERR_CUDA if the launch fails.  Asynchronous on `stream`.
+ */
+pa_status pa_hbm_read_probe(const void* buf, int64_t bytes, void* sink, void* stream);
+
+/*
  * Read and clear the device error word that kernels set when they skip an
  * out-of-range block id or slot (PA_ERR_OUT_OF_RANGE) or give up a bounded
  * wait (PA_ERR_TIMEOUT).  Synchronises `stream` first.  Returns PA_OK when no

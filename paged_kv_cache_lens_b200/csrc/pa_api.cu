@@ -516,6 +516,14 @@ pa_status pa_swap_blocks(void* dst_k, void* dst_v, const void* src_k, const void
   return PA_OK;
 }
 
+pa_status pa_hbm_read_probe(const void* buf, int64_t bytes, void* sink, void* stream) {
+  if (bytes < 0 || bytes % 16 != 0 || !sink || !aligned(sink, 4)) return PA_ERR_INVALID_ARG;
+  if (bytes > 0 && (!buf || !aligned(buf, 16))) return PA_ERR_INVALID_ARG;
+  cudaError_t e = launch_hbm_read_probe(buf, bytes, static_cast<uint32_t*>(sink),
+                                        static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : cuda_fail(e, "hbm_read_probe launch");
+}
+
 pa_status pa_device_error(void* stream) {
   cudaError_t e;
   unsigned v = read_and_clear_error_word(static_cast<cudaStream_t>(stream), &e);

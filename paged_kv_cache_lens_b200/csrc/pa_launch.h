@@ -100,6 +100,10 @@ struct MovePairs {
 cudaError_t launch_move_blocks(void* dst_k, void* dst_v, const void* src_k, const void* src_v,
                                const int64_t* host_mapping, int64_t num_pairs,
                                int64_t block_bytes, cudaStream_t stream);
+// Read-only HBM stream over `bytes` (a multiple of 16) at `buf` (16-byte
+// aligned): *sink = XOR of all 32-bit words.
+cudaError_t launch_hbm_read_probe(const void* buf, int64_t bytes, uint32_t* sink,
+                                  cudaStream_t stream);
 cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* mapping,
                                int64_t num_pairs, int64_t block_bytes, int32_t num_blocks,
                                cudaStream_t stream);

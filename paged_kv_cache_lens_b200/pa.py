@@ -85,6 +85,8 @@ def load_library(path: str = LIB_PATH):
     lib.pa_copy_blocks.restype = E
     lib.pa_swap_blocks.argtypes = [P, P, P, P, D, i64, i64, P, i64, P]
     lib.pa_swap_blocks.restype = E
+    lib.pa_hbm_read_probe.argtypes = [P, i64, P, P]
+    lib.pa_hbm_read_probe.restype = E
     if path == LIB_PATH:
         _lib = lib
     return lib
@@ -238,6 +240,14 @@ def pa_varlen(out: torch.Tensor, q: torch.Tensor, cu_seqlens_q: torch.Tensor,
     else:
         st = lib.pa_varlen_ex(*args, opts, _ptr(workspace), wbytes, _stream(stream))
         _check(st, "pa_varlen_ex")
+
+
+def pa_hbm_read_probe(buf: torch.Tensor, sink: torch.Tensor, stream=None) -> None:
+    """Stream `buf` (contiguous, device) once with read-only loads; sink (a
+    device int32 of one element) receives the XOR of its 32-bit words."""
+    st = load_library().pa_hbm_read_probe(_ptr(buf), buf.numel() * buf.element_size(),
+                                          _ptr(sink), _stream(stream))
+    _check(st, "pa_hbm_read_probe")
 
 
 def pa_device_error(stream=None) -> int:
