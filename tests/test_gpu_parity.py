@@ -128,6 +128,28 @@ def test_decode_fp8_pool(oracle, D, q_dtype):
         _run_small(oracle, W, out_dtype)
 
 
+@pytest.mark.parametrize("D", [128, 256])
+@pytest.mark.parametrize("q_dtype", [wl.BF16, wl.F16])
+def test_decode_fp8_query_dynamic_range(oracle, D, q_dtype):
+    """E4M3 pool: the query enters QK^T as E4M3 hi + lo parts of q * 2^e, one
+    power of two per head.  Heads whose elements span 2^-12 .. 2^4, an
+    all-zero head, a head of tiny values and a head with one element near
+    the 16-bit formats' 900 still match the oracle."""
+    W = wl.build_workload("fp8q", 350 + D, np.ones(4, np.int64), [9, 200, 777, 1500], 8, 2, D,
+                          dtype=q_dtype, kv_dtype=wl.FP8_E4M3)
+    rng = np.random.default_rng(D + q_dtype)
+    q = rng.standard_normal((W.total_q, 8, D)).astype(np.float32)
+    q *= np.exp2(rng.uniform(-12, 4, size=q.shape)).astype(np.float32)
+    q[:, 1, :] = 0.0
+    q[:, 2, :] *= np.float32(2.0 ** -20)
+    q[:, 5, 7] = 900.0
+    if q_dtype == wl.BF16:
+        W.q = wl.f32_to_bf16_bits(q)
+    else:
+        W.q = q.astype(np.float16).view(np.uint16)
+    _run_small(oracle, W, F32)
+
+
 def test_decode_f16(oracle):
     W = wl.build_workload("f16", 77, np.ones(5, np.int64), [3, 40, 300, 700, 1500], 32, 8, 128,
                           dtype=wl.F16)
