@@ -482,37 +482,81 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
 }
 
 // Compact list of (request, query tile) items of the q_len >= 2 requests,
-// heaviest tiles of each request first.  One CTA; a block-wide running scan.
-__global__ void __launch_bounds__(256)
-prefill_items_kernel(int32_t num_seqs, const int32_t* cu, int tq, int2* items, int32_t* count,
-                     int32_t capacity) {
-  __shared__ int s_scan[256];
-  __shared__ int s_base;
-  if (threadIdx.x == 0) s_base = 0;
+// ordered by the number of key tiles each visits, most first (longest
+// processing time first: the heavy CTAs start in the first wave instead of
+// forming the grid's tail).  One CTA: a histogram of item weights in shared
+// memory, a descending exclusive scan over it, then each item takes a slot in
+// its weight's range (order within one weight is arbitrary; every item
+// writes its own output rows, so the result does not depend on it).
+constexpr int kItemThreads = 1024;
+constexpr int kWeightBuckets = 4096;     // weights past the last bucket share it
+
+__device__ __forceinline__ int item_weight(const int32_t* cu, const int32_t* seqlens_k,
+                                           int32_t max_context_len, int32_t window, int tq,
+                                           int r, int qt) {
+  const int q_len = cu[r + 1] - cu[r];
+  const int kv_len = min(seqlens_k[r], max_context_len);
+  const int rows = min(tq, q_len - qt * tq);
+  const int pos0 = kv_len - q_len + qt * tq;
+  const int last = pos0 + rows - 1;
+  if (rows <= 0 || last < 0) return 0;
+  const int jlo = window > 0 ? max(0, pos0 - window + 1) / kBN : 0;
+  return min(last / kBN + 1 - jlo, kWeightBuckets - 1);
+}
+
+__global__ void __launch_bounds__(kItemThreads)
+prefill_items_kernel(int32_t num_seqs, const int32_t* cu, const int32_t* seqlens_k,
+                     int32_t max_context_len, int32_t window, int tq, int2* items,
+                     int32_t* count, int32_t capacity) {
+  __shared__ int s_hist[kWeightBuckets];
+  __shared__ int s_part[kItemThreads];
+  for (int i = threadIdx.x; i < kWeightBuckets; i += kItemThreads) s_hist[i] = 0;
   __syncthreads();
-  for (int r0 = 0; r0 < num_seqs; r0 += 256) {
-    const int r = r0 + threadIdx.x;
-    int n = 0;
-    if (r < num_seqs) {
-      const int ql = cu[r + 1] - cu[r];
-      n = ql >= 2 ? (ql + tq - 1) / tq : 0;
-    }
-    s_scan[threadIdx.x] = n;
+  // ---- histogram of item weights
+  for (int r = threadIdx.x; r < num_seqs; r += kItemThreads) {
+    const int ql = cu[r + 1] - cu[r];
+    if (ql < 2) continue;
+    for (int qt = 0; qt < (ql + tq - 1) / tq; ++qt)
+      atomicAdd(&s_hist[item_weight(cu, seqlens_k, max_context_len, window, tq, r, qt)], 1);
+  }
+  __syncthreads();
+  // ---- descending exclusive scan: bucket w starts after every heavier item.
+  // Thread t owns buckets kWeightBuckets-1-4t .. -3 (4 per thread, heaviest first).
+  constexpr int kPer = kWeightBuckets / kItemThreads;
+  int mine[kPer], sum = 0;
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    mine[k] = s_hist[kWeightBuckets - 1 - (kPer * threadIdx.x + k)];
+    sum += mine[k];
+  }
+  s_part[threadIdx.x] = sum;
+  __syncthreads();
+  for (int off = 1; off < kItemThreads; off <<= 1) {      // inclusive Hillis-Steele scan
+    const int v = threadIdx.x >= off ? s_part[threadIdx.x - off] : 0;
     __syncthreads();
-    for (int off = 1; off < 256; off <<= 1) {      // inclusive Hillis-Steele scan
-      const int v = threadIdx.x >= off ? s_scan[threadIdx.x - off] : 0;
-      __syncthreads();
-      s_scan[threadIdx.x] += v;
-      __syncthreads();
-    }
-    const int start = s_base + s_scan[threadIdx.x] - n;
-    for (int k = 0; k < n; ++k)
-      if (start + k < capacity) items[start + k] = make_int2(r, n - 1 - k);
-    __syncthreads();
-    if (threadIdx.x == 255) s_base += s_scan[255];
+    s_part[threadIdx.x] += v;
     __syncthreads();
   }
-  if (threadIdx.x == 0) *count = min(s_base, capacity);
+  int base = s_part[threadIdx.x] - sum;
+  const int total = s_part[kItemThreads - 1];
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    s_hist[kWeightBuckets - 1 - (kPer * threadIdx.x + k)] = base;   // next free slot
+    base += mine[k];
+  }
+  __syncthreads();
+  // ---- scatter
+  for (int r = threadIdx.x; r < num_seqs; r += kItemThreads) {
+    const int ql = cu[r + 1] - cu[r];
+    if (ql < 2) continue;
+    for (int qt = 0; qt < (ql + tq - 1) / tq; ++qt) {
+      const int slot =
+          atomicAdd(&s_hist[item_weight(cu, seqlens_k, max_context_len, window, tq, r, qt)], 1);
+      if (slot < capacity) items[slot] = make_int2(r, qt);
+    }
+  }
+  if (threadIdx.x == 0) *count = min(total, capacity);
 }
 
 template <bool BF16, int G>
@@ -563,9 +607,9 @@ cudaError_t launch_paged_prefill(const AttnArgs& a, const CUtensorMap& kmap,
                                  const CUtensorMap& vmap, const CUtensorMap& qmap,
                                  int32_t capacity, cudaStream_t stream) {
   const int tq = 128 / a.group;
-  prefill_items_kernel<<<1, 256, 0, stream>>>(a.num_seqs, a.cu_seqlens_q, tq,
-                                              const_cast<int2*>(a.pf_items),
-                                              const_cast<int32_t*>(a.pf_count), capacity);
+  prefill_items_kernel<<<1, kItemThreads, 0, stream>>>(
+      a.num_seqs, a.cu_seqlens_q, a.seqlens_k, a.max_context_len, a.window, tq,
+      const_cast<int2*>(a.pf_items), const_cast<int32_t*>(a.pf_count), capacity);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return a.kv_dtype == 1 ? launch_prefill_g<true>(a, kmap, vmap, qmap, capacity, stream)
