@@ -526,11 +526,15 @@ def _oracle_sample(W, n_seqs, threads):
 
 
 def mixed_split(torch, pa, W, args, dev, stream, q, bt, sk, out, kc, vc, ks, vs, slopes,
-                iters=50):
+                iters=30):
     """A mixed step whose leading requests are single-row decodes and the rest
     prefill chunks: each part through pa_varlen on its own (same pools, same
-    rows), CUDA events over `iters` calls.  Decode rows report KV GB/s, chunks
-    algorithmic TFLOP/s."""
+    rows), CUDA events around each of `iters` calls with the L2 flushed before
+    each by a 512 MiB read sweep (clean lines: no write-back lands inside the
+    timed call), as the full step leaves it.  Decode rows report KV GB/s,
+    chunks algorithmic TFLOP/s."""
+    flush = torch.ones(128 << 20, dtype=torch.int32, device=dev)
+    sink = torch.zeros(1, dtype=torch.int32, device=dev)
     ql = W.q_lens
     nd = 0
     while nd < W.num_seqs and ql[nd] == 1:
@@ -557,14 +561,17 @@ def mixed_split(torch, pa, W, args, dev, stream, q, bt, sk, out, kc, vc, ks, vs,
         for _ in range(3):
             call()
         torch.cuda.synchronize(dev)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(iters):
-            call()
-        b.record(stream)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(iters)]
+        with torch.cuda.stream(stream):
+            for a, b in evs:
+                pa.pa_hbm_read_probe(flush, sink, stream)
+                a.record(stream)
+                call()
+                b.record(stream)
         torch.cuda.synchronize(dev)
-        ms = a.elapsed_time(b) / iters
-        part = {"requests": r1 - r0, "rows": q1 - q0, "ms": round(ms, 5)}
+        ms = float(np.mean([a.elapsed_time(b) for a, b in evs]))
+        part = {"requests": r1 - r0, "rows": q1 - q0, "ms": round(ms, 5), "l2": "flushed"}
         if name == "decode_rows":
             kv = int(vis[r0:r1].sum()) * per_tok
             part.update(kv_bytes=kv, kv_gbs=round(kv / (ms * 1e-3) / 1e9, 1))
