@@ -185,13 +185,20 @@ size_t pa_varlen_workspace_size(int32_t num_seqs, int32_t total_q, int32_t num_q
                                 int32_t head_dim, int32_t max_context_len);
 
 /*
- * Packed mixed prefill/decode attention.  Request r owns query rows
+ * Packed mixed prefill/decode attention ("推理优化与服务：从 PagedAttention 到
+ * 分离式部署", 最新进展: the unified step packs every scheduled query token
+ * with cu_seqlens; "PagedAttention 与 Continuous Batching", §4.2: chunked
+ * prefill shares a step with decodes).  Request r owns query rows
  * cu_seqlens_q[r] .. cu_seqlens_q[r+1]-1 (q_len_r rows) and seqlens_k[r] keys
  * (kv_len_r = cached + this step's new tokens, the new ones already written by
  * pa_reshape_and_cache).  Row i of request r sits at absolute position
  * kv_len_r - q_len_r + i and attends keys 0 .. kv_len_r - q_len_r + i
  * (causal mask aligned to the bottom right).  Rows with no visible key yield
  * zeros.  q_len 1 rows are decode rows; longer ones are prefill chunks.
+ * Chunks run on the tensor-core chunk kernel when the pool is bf16/f16 with
+ * head_dim 128, q has the pool's type, the GQA group is 1, 2, 4 or 8 and out
+ * is 16-byte aligned; otherwise every row runs on the decode kernel.  Either
+ * way the result is the same attention.
  *
  * out, q       : device [total_q][num_q_heads][head_dim].
  * cu_seqlens_q : device int32 [num_seqs + 1], non-decreasing, cu[0] = 0,

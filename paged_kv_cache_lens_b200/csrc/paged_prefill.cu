@@ -23,10 +23,10 @@
 // Warp roles: 8 softmax warps in two groups of four that take alternate key
 // tiles (one thread per tile row, all 128 columns); a group passes the row
 // maxima it used to the other through shared memory, so the exponentials of
-// one group overlap the TMEM loads, maxima and stores of the other.  4 TMA
-// producer warps (paged K/V tiles are gathered 16 tokens at a time), 1 warp
-// that allocates TMEM and issues the MMAs from one thread.  S/P live in three
-// TMEM buffers: S runs up to two tiles ahead of PV.
+// one group overlap the TMEM loads, maxima and stores of the other.  2 TMA
+// producer warps (K and V; paged tiles gathered 16 tokens at a time), 1 warp
+// that allocates TMEM and issues the MMAs (one lane elected per instruction).
+// S/P live in three TMEM buffers: S runs up to two tiles ahead of PV.
 #include "pa_device.cuh"
 #include "pa_launch.h"
 
