@@ -120,3 +120,37 @@ def test_host_validation_rejects_before_any_launch(lib):
                          ctypes.byref(desc), fake, 8, 0.125, None, 0, None) == 3
     assert lib.pa_varlen(fake, 0, fake, 0, 10, 2, 2, fake, fake, 200, 100, fake, fake,
                          ctypes.byref(desc), fake, 8, 0.125, None, 0, None) == 1
+
+
+def test_block_ops_and_probe_validation(lib):
+    """Host-side checks of the block operations, the options struct and the
+    read probe: each case fails (or succeeds with no work) before any launch."""
+    import numpy as np
+    P = ctypes.c_void_p
+    fake = P(0x10000)
+    desc = _desc()
+    # copy_blocks: negative count, no pairs (a no-op), missing mapping, f32 pool,
+    # blocks that are not a whole number of 16-byte units
+    assert lib.pa_copy_blocks(fake, fake, ctypes.byref(desc), fake, -1, None) == 1
+    assert lib.pa_copy_blocks(fake, fake, ctypes.byref(desc), fake, 0, None) == 0
+    assert lib.pa_copy_blocks(fake, fake, ctypes.byref(desc), None, 3, None) == 1
+    assert lib.pa_copy_blocks(fake, fake, ctypes.byref(_desc(kv_dtype=pa.PA_F32)), fake, 3,
+                              None) == 2
+    odd = _desc(kv_dtype=pa.PA_FP8_E4M3, head_dim=1, block_size=8, num_kv_heads=1)
+    assert lib.pa_copy_blocks(fake, fake, ctypes.byref(odd), fake, 3, None) == 1
+    # swap_blocks: a pair outside either pool is caught on the host
+    m = np.array([[0, 1], [5, 2]], np.int64)
+    mp = m.ctypes.data_as(P)
+    assert lib.pa_swap_blocks(fake, fake, fake, fake, ctypes.byref(desc), 4, 8, mp, 2, None) == 1
+    assert lib.pa_swap_blocks(fake, fake, fake, fake, ctypes.byref(desc), 8, 2, mp, 2, None) == 1
+    assert lib.pa_swap_blocks(fake, fake, fake, fake, ctypes.byref(desc), 8, 8, mp, 0, None) == 0
+    assert lib.pa_swap_blocks(fake, fake, fake, fake, ctypes.byref(desc), 8, 8, mp, -1, None) == 1
+    # options: ALiBi slopes must be a 4-byte aligned float array
+    opts = pa.pa_attn_options(window=0, alibi_slopes=0x10002)
+    assert lib.pa_decode_ex(fake, 0, fake, 0, 4, 2, fake, fake, ctypes.byref(desc), fake, 8, fake,
+                            100, 0.125, 0, ctypes.byref(opts), None, 0, None) == 1
+    # read probe: sizes in 16-byte units, aligned buffer and sink
+    assert lib.pa_hbm_read_probe(fake, 24, fake, None) == 1
+    assert lib.pa_hbm_read_probe(fake, -16, fake, None) == 1
+    assert lib.pa_hbm_read_probe(fake, 32, None, None) == 1
+    assert lib.pa_hbm_read_probe(P(0x10008), 32, fake, None) == 1
