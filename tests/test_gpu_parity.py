@@ -281,6 +281,22 @@ def test_full_size_decode_sampled(oracle, cfg):
     ph = np.tile(np.arange(W.num_q_heads), len(rows))
     want = oracle_attention(oracle, W, kc, vc, pairs=(pr, ph), num_threads=8)
     assert_close(got[pr, ph], want, W, W.out_dtype, W.name)
+    _assert_visible_slots_equal(d, W, kc, vc, rows)
+
+
+def _assert_visible_slots_equal(d, W, kc, vc, rows):
+    """Every slot a sampled request's attention reads holds, bit for bit, what
+    the oracle's cache write put there (full-size pools, written in pieces by
+    pa_reshape_and_cache)."""
+    reqs = sorted({int(np.searchsorted(W.cu_seqlens_q, r, side="right") - 1) for r in rows})
+    for rq in reqs:
+        t = np.arange(int(W.seqlens_k[rq]))
+        blk = W.block_tables[rq, t // W.block_size].astype(np.int64)
+        off = t % W.block_size
+        idx = torch.from_numpy(blk).cuda(), torch.from_numpy(off).cuda()
+        for dev_pool, host_pool in ((d.k_cache, kc), (d.v_cache, vc)):
+            got = _pool_bits(dev_pool[idx[0], :, idx[1], :])        # [L, Hkv, D]
+            assert np.array_equal(got, host_pool[blk, :, off, :]), f"request {rq}"
 
 
 def test_full_size_mixed_step_sampled(oracle):
@@ -305,6 +321,7 @@ def test_full_size_mixed_step_sampled(oracle):
     ph = np.tile(heads, len(rows))
     want = oracle_attention(oracle, W, kc, vc, pairs=(pr, ph), num_threads=8)
     assert_close(got[pr, ph], want, W, W.out_dtype, W.name)
+    _assert_visible_slots_equal(d, W, kc, vc, rows)
 
 
 # ---------------------------------------------------------------- errors
