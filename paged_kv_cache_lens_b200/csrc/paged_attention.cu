@@ -606,15 +606,13 @@ cudaError_t launch_typed(const AttnArgs& a, const CUtensorMap& kmap, const CUten
   constexpr int NSTAGE = 2;
   using S = Smem<KVT, D, GT, NSTAGE>;
   auto kern = paged_attn_kernel<KVT, Q_BF16, D, GT, NSTAGE>;
-  static bool configured = false;   // per instantiation; idempotent if raced
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         S::kTotal);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
   const int64_t grid = static_cast<int64_t>(a.rows) * a.num_kv_heads * a.max_parts;
   if (grid == 0) return cudaSuccess;
+  // the shared-memory limit is a per-device setting of the function: set it
+  // for the current device on every launch (a host-side call)
+  cudaError_t se =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kTotal);
+  if (se != cudaSuccess) return se;
   kern<<<static_cast<unsigned>(grid), kThreads, S::kTotal, stream>>>(a, kmap, vmap);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

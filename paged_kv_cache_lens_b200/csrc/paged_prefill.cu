@@ -563,15 +563,13 @@ template <bool BF16, int G>
 cudaError_t launch_prefill_typed(const AttnArgs& a, const CUtensorMap& k, const CUtensorMap& v,
                                  const CUtensorMap& q, int capacity, cudaStream_t s) {
   auto kern = paged_prefill_kernel<BF16, G>;
-  static bool configured = false;   // one flag per instantiation
-  if (!configured) {
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
   const int64_t grid = static_cast<int64_t>(capacity) * a.num_kv_heads;
   if (grid == 0) return cudaSuccess;
+  // the shared-memory limit is a per-device setting of the function: set it
+  // for the current device on every launch (a host-side call)
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  if (e != cudaSuccess) return e;
   kern<<<static_cast<unsigned>(grid), kPfThreads, kSmemBytes, s>>>(a, k, v, q);
   return cudaGetLastError();
 }
