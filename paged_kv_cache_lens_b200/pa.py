@@ -115,6 +115,28 @@ def dtype_code(t: torch.dtype, fp8_if_byte: bool = False) -> int:
     raise ValueError(f"no libpa dtype for {t}")
 
 
+def _need(t: Optional[torch.Tensor], name: str, dtype=None, rows_strided: bool = False,
+          pinned_ok: bool = False) -> None:
+    """The library reads every tensor through a raw pointer with a fixed
+    layout: reject, before any launch, what it would misread (a host tensor,
+    a non-contiguous view, the wrong element type)."""
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name}: expected {dtype}, got {t.dtype}")
+    if rows_strided:
+        # [rows, ...] with any row stride, each row itself contiguous
+        if t.dim() < 2 or (t.shape[0] > 0 and not t[0].is_contiguous()):
+            raise ValueError(f"{name}: each row must be contiguous")
+    elif not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if t.device.type != "cuda" and not (pinned_ok and t.is_pinned()):
+        where = "CUDA or pinned host memory" if pinned_ok else "a CUDA tensor"
+        raise ValueError(f"{name}: must be {where} (got {t.device})")
+
+
 def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
@@ -155,7 +177,15 @@ def pa_reshape_and_cache(key: torch.Tensor, value: torch.Tensor, slot_mapping: t
                          v_scale=None, stream=None) -> None:
     """key/value: [T, Hkv, D] (rows may be strided, e.g. views into a fused QKV
     buffer); slot_mapping: int64 [T]; pools [NB, Hkv, 16, D]."""
-    assert key.stride() == value.stride() and key.stride(-1) == 1
+    _need(key, "key", rows_strided=True)
+    _need(value, "value", rows_strided=True)
+    if key.shape != value.shape or key.stride() != value.stride():
+        raise ValueError("key and value must have the same shape and strides")
+    _need(slot_mapping, "slot_mapping", torch.int64)
+    _need(k_cache, "k_cache")
+    _need(v_cache, "v_cache")
+    _need(k_scale, "k_scale", torch.float32)
+    _need(v_scale, "v_scale", torch.float32)
     T = key.shape[0]
     desc = cache_desc(k_cache, k_scale, v_scale)
     st = load_library().pa_reshape_and_cache(
@@ -198,6 +228,13 @@ def pa_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache
               alibi_slopes: Optional[torch.Tensor] = None) -> None:
     """out/q: [B, Hq, D]; block_tables int32 [B, max_blocks]; context_lens int32 [B].
     window / alibi_slopes select pa_decode_ex's sliding window and ALiBi."""
+    for t, n in ((out, "out"), (q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"),
+                 (workspace, "workspace")):
+        _need(t, n)
+    _need(block_tables, "block_tables", torch.int32)
+    _need(context_lens, "context_lens", torch.int32)
+    for t, n in ((k_scale, "k_scale"), (v_scale, "v_scale"), (alibi_slopes, "alibi_slopes")):
+        _need(t, n, torch.float32)
     B, hq, d = q.shape
     lib = load_library()
     need = lib.pa_decode_workspace_size(B, hq, d, max_context_len, partition_size)
@@ -223,6 +260,14 @@ def pa_varlen(out: torch.Tensor, q: torch.Tensor, cu_seqlens_q: torch.Tensor,
               stream=None, window: int = 0, alibi_slopes: Optional[torch.Tensor] = None) -> None:
     """out/q: [total_q, Hq, D]; cu_seqlens_q int32 [S+1]; seqlens_k int32 [S].
     window / alibi_slopes select pa_varlen_ex's sliding window and ALiBi."""
+    for t, n in ((out, "out"), (q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"),
+                 (workspace, "workspace")):
+        _need(t, n)
+    for t, n in ((cu_seqlens_q, "cu_seqlens_q"), (seqlens_k, "seqlens_k"),
+                 (block_tables, "block_tables")):
+        _need(t, n, torch.int32)
+    for t, n in ((k_scale, "k_scale"), (v_scale, "v_scale"), (alibi_slopes, "alibi_slopes")):
+        _need(t, n, torch.float32)
     total_q, hq, d = q.shape
     S = seqlens_k.shape[0]
     lib = load_library()
@@ -245,6 +290,8 @@ def pa_varlen(out: torch.Tensor, q: torch.Tensor, cu_seqlens_q: torch.Tensor,
 def pa_hbm_read_probe(buf: torch.Tensor, sink: torch.Tensor, stream=None) -> None:
     """Stream `buf` (contiguous, device) once with read-only loads; sink (a
     device int32 of one element) receives the XOR of its 32-bit words."""
+    _need(buf, "buf")
+    _need(sink, "sink")
     st = load_library().pa_hbm_read_probe(_ptr(buf), buf.numel() * buf.element_size(),
                                           _ptr(sink), _stream(stream))
     _check(st, "pa_hbm_read_probe")
@@ -258,6 +305,9 @@ def pa_device_error(stream=None) -> int:
 def pa_copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, block_mapping: torch.Tensor,
                    stream=None) -> None:
     """block_mapping: device int64 [n, 2] of (src, dst) block ids."""
+    _need(k_cache, "k_cache")
+    _need(v_cache, "v_cache")
+    _need(block_mapping, "block_mapping", torch.int64)
     desc = cache_desc(k_cache)
     n = block_mapping.shape[0]
     st = load_library().pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), ctypes.byref(desc),
@@ -270,6 +320,8 @@ def pa_swap_blocks(dst_k: torch.Tensor, dst_v: torch.Tensor, src_k: torch.Tensor
     """Pools on the device or in pinned host memory; block_mapping: host
     (src, dst) pairs (anything numpy can turn into int64 [n, 2])."""
     import numpy as np
+    for t, n in ((dst_k, "dst_k"), (dst_v, "dst_v"), (src_k, "src_k"), (src_v, "src_v")):
+        _need(t, n, pinned_ok=True)
     pairs = np.ascontiguousarray(np.asarray(block_mapping, dtype=np.int64).reshape(-1, 2))
     desc = cache_desc(src_k)
     st = load_library().pa_swap_blocks(
