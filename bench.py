@@ -407,7 +407,9 @@ def run_native(args):
     gbs = by["kv"] * world / (ms * 1e-3) / 1e9
     attn_gbs = by["attention"] / (attn_ms * 1e-3) / 1e9
     seq_steps = W.num_seqs * world / (ms * 1e-3)
-    traffic = recorded_traffic(W)
+    # the table holds captures of the full-size workloads without window or ALiBi
+    plain = args.batch is None and not args.window and not args.alibi
+    traffic = recorded_traffic(W) if plain else None
     line = {
         "metric": METRIC,
         "value": round(gbs, 1),
@@ -474,16 +476,21 @@ def recorded_traffic(W):
             for line in f:
                 parts = line.split()
                 if len(parts) == 3 and parts[0] == W.name and not line.startswith("#"):
-                    return int(parts[2]) if parts[1] == kernel_sha() else None
+                    return int(parts[2]) if parts[1] == kernel_sha(W) else None
     except OSError:
         return None
     return None
 
 
-def kernel_sha():
+def kernel_sha(W=None):
+    """Hash of the kernel sources a workload's attention call runs: the decode
+    kernel's, plus the chunk kernel's for a step with prefill chunks."""
     import hashlib
     h = hashlib.sha256()
-    for name in ("paged_attention.cu", "pa_device.cuh", "pa_launch.h"):
+    names = ["paged_attention.cu", "pa_device.cuh", "pa_launch.h"]
+    if W is not None and not W.decode:
+        names.append("paged_prefill.cu")
+    for name in names:
         with open(os.path.join(ROOT, "paged_kv_cache_lens_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]

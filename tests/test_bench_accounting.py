@@ -41,3 +41,21 @@ def test_window_bytes_count_visible_keys_only():
     per_tok = 2 * 2 * 128 * 2
     assert bench.algorithmic_bytes(W, 64)["kv_logical"] == (64 + 10) * per_tok
     assert np.array_equal(bench.visible_keys(W, 64), [64, 10])
+
+
+def test_traffic_is_used_only_for_the_sources_it_was_taken_on(monkeypatch):
+    """profiles/traffic.txt holds DRAM bytes keyed by the hash of the kernel
+    sources a workload runs; another hash yields no traffic figure."""
+    W2, W4 = wl.config(2, batch=4), wl.config(4, batch=8)
+    assert bench.kernel_sha(W2) == bench.kernel_sha()          # decode kernel sources
+    assert bench.kernel_sha(W4) != bench.kernel_sha(W2)        # plus the chunk kernel's
+    table = {}
+    for line in open(bench.os.path.join(bench.ROOT, "profiles", "traffic.txt")):
+        if line.strip() and not line.startswith("#"):
+            name, sha, nbytes = line.split()
+            table[name] = (sha, int(nbytes))
+    sha, nbytes = table[W2.name]
+    monkeypatch.setattr(bench, "kernel_sha", lambda W=None: sha)
+    assert bench.recorded_traffic(W2) == nbytes
+    monkeypatch.setattr(bench, "kernel_sha", lambda W=None: "0" * 16)
+    assert bench.recorded_traffic(W2) is None
