@@ -1,7 +1,7 @@
 """A NumPy model of the chunk kernel's arithmetic (CPU only): 128-key tiles,
 a running maximum raised only when a tile exceeds it by 2^8, P = 2^(x - m)
 entering PV as a bf16 hi + lo pair, fp32 sums.  It pins the precision claim
-behind the hi + lo split against the fp64 oracle: with the pair the error is
+behind the hi + lo split against the exact fp64 result: with the pair the error is
 far inside the 2e-3 bound; with P as one bf16 value a row with a few large
 values leaves it."""
 import numpy as np
