@@ -4,9 +4,13 @@
 One step = the whole path over one batch: write the step's new K/V rows into
 the paged pool (pa_reshape_and_cache), then paged attention over every
 sequence's cached context (pa_decode; pa_varlen for the mixed step).  The
-default workload is the LLaMA-13B-shaped MHA decode: 64 sequences, context
-lengths uniform in [128, 2048], 40 heads of dimension 128, bf16, 16-token
-blocks in a 12000-block pool.
+default (headline) workload is the Llama-3-8B-shaped GQA decode: 256
+sequences, context lengths lognormal (median 1000) clipped to [32, 8192], 32
+query heads over 8 KV heads of dimension 128, bf16, 16-token blocks, split-K
+partitions of 512 tokens.  After it, the same line carries a compact record
+of each other workload measured on the same contract ("configs"): the
+LLaMA-13B MHA decode, the mixed prefill/decode step (with its decode rows and
+prefill chunks timed apart) and the shared-prefix FP8 decode.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 2..5] [--impl reference]
 
@@ -35,6 +39,9 @@ from paged_kv_cache_lens_b200 import workloads as wl  # noqa: E402
 
 METRIC = "paged decode attention: achieved HBM GB/s (% of peak), sequence-steps/s/layer"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+DEFAULT_WORKLOAD = 3
+SUB_WORKLOADS = (2, 4, 5)
 CLOCK_QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -45,7 +52,7 @@ def parse_args():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", type=int, default=2, choices=[2, 3, 4, 5])
+    ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD, choices=[2, 3, 4, 5])
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--op", default="step", choices=["step", "copy_blocks", "swap_blocks"],
                     help="step: the attention step (default); copy_blocks / swap_blocks: "
@@ -57,17 +64,9 @@ def parse_args():
     ap.add_argument("--alibi", action="store_true", help="ALiBi slopes 2^(-8 i / H)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-sub", action="store_true",
+                    help="skip the compact records of the other workloads")
     return ap.parse_args()
-
-
-def peaks():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    try:
-        with open(p) as f:
-            d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
-    except (OSError, KeyError, ValueError):
-        return FALLBACK_HBM_GBS, "fallback"
 
 
 NOMINAL_HBM_GBS = 8000.0     # B200 HBM3e, nominal (context beside the measured copy peak)
@@ -252,6 +251,285 @@ def max_over_ranks(x: float, world: int) -> float:
 # the native arm
 # --------------------------------------------------------------------------
 
+TD_NAMES = {wl.F16: "float16", wl.BF16: "bfloat16", wl.F32: "float32"}
+
+
+def chunk_path(W) -> bool:
+    """Whether pa_varlen sends this step's q_len >= 2 requests to the
+    tensor-core chunk kernel (the library's rule: 16-bit KV and q of one type,
+    head_dim 128, GQA group 1, 2, 4 or 8)."""
+    g = W.num_q_heads // W.num_kv_heads
+    return (not W.decode and W.max_q_len >= 2 and W.kv_dtype in (wl.F16, wl.BF16)
+            and W.q_dtype == W.kv_dtype and W.head_dim == 128 and g in (1, 2, 4, 8))
+
+
+class DeviceWorkload:
+    """One workload resident on the GPU: the paged pools holding the cached
+    context, the step's inputs, the output and the workspace; step() is one
+    pass of the whole path (cache write of the new rows, then attention)."""
+
+    def __init__(self, torch, pa, W, dev, window=0, alibi=False):
+        self.torch, self.pa, self.W, self.dev = torch, pa, W, dev
+        self.window = window
+        TD = {k: getattr(torch, v) for k, v in TD_NAMES.items()}
+        self.TD = TD
+        shape = (W.num_blocks, W.num_kv_heads, W.block_size, W.head_dim)
+        if W.kv_dtype == wl.FP8_E4M3:
+            self.kc = torch.zeros(shape, dtype=torch.uint8, device=dev)
+            self.vc = torch.zeros(shape, dtype=torch.uint8, device=dev)
+            self.ks = torch.from_numpy(W.k_scale).to(dev)
+            self.vs = torch.from_numpy(W.v_scale).to(dev)
+        else:
+            self.kc = torch.zeros(shape, dtype=TD[W.kv_dtype], device=dev)
+            self.vc = torch.zeros(shape, dtype=TD[W.kv_dtype], device=dev)
+            self.ks = self.vs = None
+        self.stream = torch.cuda.current_stream(dev)
+        # cached context (set-up, untimed)
+        chunk = 1 << 18
+        for s in range(0, len(W.prefill_slots), chunk):
+            e = min(len(W.prefill_slots), s + chunk)
+            pa.pa_reshape_and_cache(self.to_dev(W.prefill_k[s:e], W.src_dtype),
+                                    self.to_dev(W.prefill_v[s:e], W.src_dtype),
+                                    torch.from_numpy(W.prefill_slots[s:e]).to(dev),
+                                    self.kc, self.vc, self.ks, self.vs)
+        torch.cuda.synchronize(dev)
+        # step inputs resident in HBM
+        self.q = self.to_dev(W.q, W.q_dtype)
+        self.nk = self.to_dev(W.new_k, W.src_dtype)
+        self.nv = self.to_dev(W.new_v, W.src_dtype)
+        self.slots = torch.from_numpy(W.new_slots).to(dev)
+        self.bt = torch.from_numpy(W.block_tables).to(dev)
+        self.sk = torch.from_numpy(W.seqlens_k).to(dev)
+        self.cu = torch.from_numpy(W.cu_seqlens_q).to(dev)
+        self.out = torch.empty((W.total_q, W.num_q_heads, W.head_dim), dtype=TD[W.out_dtype],
+                               device=dev)
+        if W.decode:
+            nws = pa.pa_decode_workspace_size(W.num_seqs, W.num_q_heads, W.head_dim,
+                                              W.max_context_len, W.partition_size)
+        else:
+            nws = pa.pa_varlen_workspace_size(W.num_seqs, W.total_q, W.num_q_heads,
+                                              W.head_dim, W.max_context_len)
+        self.partials = nws > 0 and (W.decode or self._varlen_partials())
+        self.ws = torch.empty(max(nws, 256), dtype=torch.uint8, device=dev)
+        self.slopes = None
+        if alibi:
+            self.slopes = torch.tensor([2.0 ** (-8.0 * (i + 1) / W.num_q_heads)
+                                        for i in range(W.num_q_heads)], dtype=torch.float32,
+                                       device=dev)
+
+    def _varlen_partials(self):
+        W = self.W
+        rows = max(W.num_seqs, W.total_q)
+        ps = 512
+        while ps > 128 and rows * W.num_q_heads * (-(-W.max_context_len // ps)) < 2048:
+            ps //= 2
+        return -(-W.max_context_len // ps) > 1
+
+    def to_dev(self, a, dt):
+        t = self.torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(self.dev)
+        return t.view(self.TD[dt])
+
+    def attend(self, q, bt, sk, cu, out, stream=None):
+        W, pa = self.W, self.pa
+        stream = self.stream if stream is None else stream
+        if W.decode:
+            pa.pa_decode(out, q, self.kc, self.vc, bt, sk, W.max_context_len, W.scale, self.ks,
+                         self.vs, W.partition_size, self.ws, stream, window=self.window,
+                         alibi_slopes=self.slopes)
+        else:
+            pa.pa_varlen(out, q, cu, sk, W.max_q_len, W.max_context_len, self.kc, self.vc, bt,
+                         W.scale, self.ks, self.vs, self.ws, stream, window=self.window,
+                         alibi_slopes=self.slopes)
+
+    def write_new(self, nk, nv, slots, stream=None):
+        self.pa.pa_reshape_and_cache(nk, nv, slots, self.kc, self.vc, self.ks, self.vs,
+                                     self.stream if stream is None else stream)
+
+    def step(self):
+        self.write_new(self.nk, self.nv, self.slots)
+        self.attend(self.q, self.bt, self.sk, self.cu, self.out)
+
+    def launches_per_step(self) -> int:
+        """Kernels of this library one step launches: the cache write, then
+        attention (decode kernel; plus the work-list and chunk kernels for a
+        step with prefill chunks, or the row-map kernel without them), plus
+        the partition merge when some row spans several partitions."""
+        W = self.W
+        n = 1 + 1 + (1 if self.partials else 0)
+        if not W.decode:
+            n += 2 if chunk_path(W) else 1
+        return n
+
+    def time_steps(self, steps, warmup, world=1, clocks=None):
+        """Device time of `steps` whole steps (CUDA events on the launching
+        stream), and the mean duration of the attention call inside them."""
+        torch = self.torch
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(warmup):
+            self.step()
+        barrier(world)
+        torch.cuda.synchronize(self.dev)
+        if clocks:
+            clocks.mark_start()
+        t0.record(self.stream)
+        for i in range(steps):
+            self.write_new(self.nk, self.nv, self.slots)
+            ev[i][0].record(self.stream)
+            self.attend(self.q, self.bt, self.sk, self.cu, self.out)
+            ev[i][1].record(self.stream)
+        t1.record(self.stream)
+        torch.cuda.synchronize(self.dev)
+        if clocks:
+            clocks.mark_end()
+        barrier(world)
+        ms = max_over_ranks(t0.elapsed_time(t1) / steps, world)
+        attn = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in ev])), world)
+        assert self.pa.pa_device_error(self.stream) == 0
+        return ms, attn
+
+    def time_e2e(self, steps, warmup, world=1):
+        """The step through the public API from pinned host memory: every step
+        copies its inputs (q, new K/V rows, slots, block tables, lengths,
+        cu_seqlens) host -> device as one packed transfer and reads its output
+        back device -> host.  Transfers run on a second stream, double
+        buffered, so step i+1's inputs cross while step i computes."""
+        torch, W = self.torch, self.W
+        parts = [("q", W.q.view(np.uint8)), ("nk", W.new_k.view(np.uint8)),
+                 ("nv", W.new_v.view(np.uint8)), ("slots", W.new_slots.view(np.uint8)),
+                 ("bt", W.block_tables.view(np.uint8)), ("sk", W.seqlens_k.view(np.uint8)),
+                 ("cu", W.cu_seqlens_q.view(np.uint8))]
+        offs, n = {}, 0
+        for name, a in parts:
+            offs[name] = (n, a.nbytes)
+            n += -(-a.nbytes // 256) * 256
+        host = torch.empty(n, dtype=torch.uint8).pin_memory()
+        hv = host.numpy()
+        for name, a in parts:
+            o, b = offs[name]
+            hv[o:o + b] = np.ascontiguousarray(a).reshape(-1)
+        h_out = torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory()
+        dbuf = [torch.empty(n, dtype=torch.uint8, device=self.dev) for _ in range(2)]
+        outs = [torch.empty_like(self.out) for _ in range(2)]
+
+        def views(buf):
+            def v(name, dt, shape):
+                o, b = offs[name]
+                return buf[o:o + b].view(dt).view(shape)
+            TQ = self.TD[W.q_dtype]
+            TS = self.TD[W.src_dtype]
+            return (v("q", TQ, self.q.shape), v("nk", TS, self.nk.shape),
+                    v("nv", TS, self.nv.shape), v("slots", torch.int64, self.slots.shape),
+                    v("bt", torch.int32, self.bt.shape), v("sk", torch.int32, self.sk.shape),
+                    v("cu", torch.int32, self.cu.shape))
+        vw = [views(b) for b in dbuf]
+        cs = torch.cuda.Stream(self.dev)
+        E = lambda: torch.cuda.Event()  # noqa: E731
+        ready, consumed, drained = [E(), E()], [E(), E()], [E(), E()]
+        for e in consumed + drained:
+            e.record(self.stream)
+
+        def h2d(i):
+            b = i % 2
+            cs.wait_event(consumed[b])
+            with torch.cuda.stream(cs):
+                dbuf[b].copy_(host, non_blocking=True)
+            ready[b].record(cs)
+
+        def run(i):
+            b = i % 2
+            q, nk, nv, slots, bt, sk, cu = vw[b]
+            self.stream.wait_event(ready[b])
+            self.stream.wait_event(drained[b])
+            self.write_new(nk, nv, slots)
+            self.attend(q, bt, sk, cu, outs[b])
+            consumed[b].record(self.stream)
+            cs.wait_event(consumed[b])
+            with torch.cuda.stream(cs):
+                h_out.copy_(outs[b], non_blocking=True)
+            drained[b].record(cs)
+
+        def loop(k):
+            h2d(0)
+            for i in range(k):
+                if i + 1 < k:
+                    h2d(i + 1)
+                run(i)
+
+        loop(max(warmup, 1))
+        torch.cuda.synchronize(self.dev)
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(self.stream)
+        cs.wait_event(e0)
+        loop(steps)
+        self.stream.wait_event(drained[(steps - 1) % 2])
+        e1.record(self.stream)
+        torch.cuda.synchronize(self.dev)
+        ms = max_over_ranks(e0.elapsed_time(e1) / steps, world)
+        h2d_bytes = sum(a.nbytes for _, a in parts)
+        d2h_bytes = h_out.numel() * h_out.element_size()
+        assert self.pa.pa_device_error(self.stream) == 0
+        return ms, h2d_bytes, d2h_bytes
+
+    def free(self):
+        for k in list(vars(self)):
+            if k not in ("torch", "pa", "W", "dev", "TD"):
+                setattr(self, k, None)
+        self.torch.cuda.empty_cache()
+
+
+def peaks():
+    """Roofline denominators: the measured copy bandwidth and bf16 dense
+    rate of this machine's B200s (generated MEASURED_PEAKS.json), else the
+    recipe's fallback figures."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        hbm = float(d["hbm_gbs"])
+        bf16 = float(d.get("bf16_tflops", FALLBACK_BF16_TFLOPS))
+        return {"hbm": hbm, "bf16": bf16, "kind": "measured"}
+    except (OSError, KeyError, ValueError, TypeError):
+        return {"hbm": FALLBACK_HBM_GBS, "bf16": FALLBACK_BF16_TFLOPS, "kind": "fallback"}
+
+
+def sub_record(torch, pa, c, dev, args, pk):
+    """A compact record of reference workload c measured the same way as the
+    headline (K timed steps after W warm-up steps, CUDA events)."""
+    W = wl.config(c)
+    d = DeviceWorkload(torch, pa, W, dev)
+    clocks = ClockSampler(dev.index or 0)
+    clocks.start()
+    ms, attn_ms = d.time_steps(args.steps, args.warmup, 1, clocks)
+    clocks.stop()
+    by = algorithmic_bytes(W)
+    attn_gbs = by["attention"] / (attn_ms * 1e-3) / 1e9
+    rec = {"workload": workload_name(W), "ms_per_step": round(ms, 5),
+           "attention_ms": round(attn_ms, 5), "algorithmic_bytes": by["attention"],
+           "achieved_gbs": round(attn_gbs, 1), "frac": round(attn_gbs / pk["hbm"], 4),
+           "traffic": recorded_traffic(W),
+           "kv_gbs_per_step": round(by["kv"] / (ms * 1e-3) / 1e9, 1),
+           "seq_steps_per_s_per_layer": round(W.num_seqs / (ms * 1e-3), 1),
+           "clocks": clocks.summary()}
+    if by["kv_logical"] != by["kv"]:
+        rec["unique_kv_bytes"] = by["kv"]
+        rec["logical_kv_bytes"] = by["kv_logical"]
+        rec["logical_gbs"] = round(by["kv_logical"] / (attn_ms * 1e-3) / 1e9, 1)
+        rec["note"] = "achieved/frac count distinct KV bytes (shared prefix once)"
+    if not W.decode:
+        split = mixed_split(torch, pa, W, args, dev, d.stream, d.q, d.bt, d.sk, d.out, d.kc,
+                            d.vc, d.ks, d.vs, None)
+        if split:
+            split["decode_rows"]["frac"] = round(split["decode_rows"]["kv_gbs"] / pk["hbm"], 4)
+            split["chunks"]["frac_of_bf16_peak"] = round(
+                split["chunks"]["tflops"] / pk["bf16"], 4)
+            rec["split"] = split
+    d.free()
+    return rec
+
+
 def run_native(args):
     import torch
     from paged_kv_cache_lens_b200 import pa
@@ -259,136 +537,22 @@ def run_native(args):
     rank, world, local = dist_setup(args.gpus)
     dev = torch.device("cuda", local if world > 1 else 0)
     W = wl.config(args.workload, batch=args.batch)
-    TD = {wl.F16: torch.float16, wl.BF16: torch.bfloat16, wl.F32: torch.float32}
+    d = DeviceWorkload(torch, pa, W, dev, args.window, args.alibi)
+    stream = d.stream
 
-    def to_dev(a, dt):
-        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(TD[dt])
-
-    shape = (W.num_blocks, W.num_kv_heads, W.block_size, W.head_dim)
-    if W.kv_dtype == wl.FP8_E4M3:
-        kc = torch.zeros(shape, dtype=torch.uint8, device=dev)
-        vc = torch.zeros(shape, dtype=torch.uint8, device=dev)
-        ks = torch.from_numpy(W.k_scale).to(dev)
-        vs = torch.from_numpy(W.v_scale).to(dev)
-    else:
-        kc = torch.zeros(shape, dtype=TD[W.kv_dtype], device=dev)
-        vc = torch.zeros(shape, dtype=TD[W.kv_dtype], device=dev)
-        ks = vs = None
-    stream = torch.cuda.current_stream(dev)
-    # cached context (setup, untimed)
-    chunk = 1 << 18
-    for s in range(0, len(W.prefill_slots), chunk):
-        e = min(len(W.prefill_slots), s + chunk)
-        pa.pa_reshape_and_cache(to_dev(W.prefill_k[s:e], W.src_dtype),
-                                to_dev(W.prefill_v[s:e], W.src_dtype),
-                                torch.from_numpy(W.prefill_slots[s:e]).to(dev), kc, vc, ks, vs)
-    torch.cuda.synchronize(dev)
-
-    # step inputs resident in HBM
-    q = to_dev(W.q, W.q_dtype)
-    nk, nv = to_dev(W.new_k, W.src_dtype), to_dev(W.new_v, W.src_dtype)
-    slots = torch.from_numpy(W.new_slots).to(dev)
-    bt = torch.from_numpy(W.block_tables).to(dev)
-    sk = torch.from_numpy(W.seqlens_k).to(dev)
-    cu = torch.from_numpy(W.cu_seqlens_q).to(dev)
-    out = torch.empty((W.total_q, W.num_q_heads, W.head_dim), dtype=TD[W.out_dtype], device=dev)
-    if W.decode:
-        nws = pa.pa_decode_workspace_size(W.num_seqs, W.num_q_heads, W.head_dim,
-                                          W.max_context_len, W.partition_size)
-    else:
-        nws = pa.pa_varlen_workspace_size(W.num_seqs, W.total_q, W.num_q_heads, W.head_dim,
-                                          W.max_context_len)
-    ws = torch.empty(max(nws, 256), dtype=torch.uint8, device=dev)
-
-    slopes = None
-    if args.alibi:
-        slopes = torch.tensor([2.0 ** (-8.0 * (i + 1) / W.num_q_heads)
-                               for i in range(W.num_q_heads)], dtype=torch.float32, device=dev)
-
-    def attend(q_, bt_, sk_, cu_, out_):
-        if W.decode:
-            pa.pa_decode(out_, q_, kc, vc, bt_, sk_, W.max_context_len, W.scale, ks, vs,
-                         W.partition_size, ws, stream, window=args.window, alibi_slopes=slopes)
-        else:
-            pa.pa_varlen(out_, q_, cu_, sk_, W.max_q_len, W.max_context_len, kc, vc, bt_,
-                         W.scale, ks, vs, ws, stream, window=args.window, alibi_slopes=slopes)
-
-    def step():
-        pa.pa_reshape_and_cache(nk, nv, slots, kc, vc, ks, vs, stream)
-        attend(q, bt, sk, cu, out)
-
-    max_parts = -(-W.max_context_len // (W.partition_size or 512))
-    launches_per_step = 1 + 1 + (1 if max_parts > 1 else 0) + (0 if W.decode else 1)
-
-    # ---- device-timed region: K whole steps, attention launches timed too
-    ev_a = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # ---- device-timed region: K whole steps, attention calls timed too
     clocks = ClockSampler(local)
     clocks.start()
-    for _ in range(args.warmup):
-        step()
-    barrier(world)
-    torch.cuda.synchronize(dev)
-    clocks.mark_start()
-    t0.record(stream)
-    for i in range(args.steps):
-        pa.pa_reshape_and_cache(nk, nv, slots, kc, vc, ks, vs, stream)
-        ev_a[i][0].record(stream)
-        attend(q, bt, sk, cu, out)
-        ev_a[i][1].record(stream)
-    t1.record(stream)
-    torch.cuda.synchronize(dev)
-    clocks.mark_end()
-    barrier(world)
+    ms, attn_ms = d.time_steps(args.steps, args.warmup, world, clocks)
     clocks.stop()
-    ms_local = t0.elapsed_time(t1) / args.steps
-    attn_ms = float(np.mean([a.elapsed_time(b) for a, b in ev_a]))
-    ms = max_over_ranks(ms_local, world)
-    attn_ms = max_over_ranks(attn_ms, world)
-    assert pa.pa_device_error(stream) == 0
 
     # ---- end to end through the public API from pinned host buffers
     e2e = None
     if not args.no_e2e:
-        pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()  # noqa: E731
-        h_q = pin(W.q.view(np.int16))
-        h_k, h_v = pin(W.new_k.view(np.int16)), pin(W.new_v.view(np.int16))
-        h_slots, h_bt = pin(W.new_slots), pin(W.block_tables)
-        h_sk, h_cu = pin(W.seqlens_k), pin(W.cu_seqlens_q)
-        h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        d_q, d_k, d_v = torch.empty_like(q), torch.empty_like(nk), torch.empty_like(nv)
-        d_slots, d_bt, d_sk, d_cu = (torch.empty_like(slots), torch.empty_like(bt),
-                                     torch.empty_like(sk), torch.empty_like(cu))
-        h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_slots, h_bt, h_sk, h_cu))
-        d2h = h_out.numel() * h_out.element_size()
-
-        def e2e_step():
-            d_q.view(torch.int16).copy_(h_q, non_blocking=True)
-            d_k.view(torch.int16).copy_(h_k, non_blocking=True)
-            d_v.view(torch.int16).copy_(h_v, non_blocking=True)
-            d_slots.copy_(h_slots, non_blocking=True)
-            d_bt.copy_(h_bt, non_blocking=True)
-            d_sk.copy_(h_sk, non_blocking=True)
-            d_cu.copy_(h_cu, non_blocking=True)
-            pa.pa_reshape_and_cache(d_k, d_v, d_slots, kc, vc, ks, vs, stream)
-            attend(d_q, d_bt, d_sk, d_cu, out)
-            h_out.copy_(out, non_blocking=True)
-
-        for _ in range(args.warmup):
-            e2e_step()
-        torch.cuda.synchronize(dev)
-        barrier(world)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, world)
-        e2e = (e2e_ms, h2d, d2h)
+        e2e = d.time_e2e(args.steps, args.warmup, world)
 
     if rank != 0:
+        d.free()
         if world > 1:
             import torch.distributed as dist
             dist.destroy_process_group()
@@ -397,13 +561,16 @@ def run_native(args):
     # ---- context measured after the timed region: read-only HBM ceiling and,
     # for a mixed step, its decode rows and prefill chunks timed apart
     probe = read_probe_gbs(torch, pa, dev, stream)
+    pk = peaks()
     split = None
     if not W.decode:
-        split = mixed_split(torch, pa, W, args, dev, stream, q, bt, sk, out, kc, vc, ks, vs,
-                            slopes)
+        split = mixed_split(torch, pa, W, args, dev, stream, d.q, d.bt, d.sk, d.out, d.kc, d.vc,
+                            d.ks, d.vs, d.slopes)
+    launches = d.launches_per_step() * args.steps
+    d.free()
 
     by = algorithmic_bytes(W, args.window)
-    peak, peak_kind = peaks()
+    peak = pk["hbm"]
     gbs = by["kv"] * world / (ms * 1e-3) / 1e9
     attn_gbs = by["attention"] / (attn_ms * 1e-3) / 1e9
     seq_steps = W.num_seqs * world / (ms * 1e-3)
@@ -442,7 +609,7 @@ def run_native(args):
             "bound": "hbm", "kernel": "pa_decode" if W.decode else "pa_varlen",
             "achieved": round(attn_gbs, 1), "peak": peak, "unit": "GB/s",
             "frac": round(attn_gbs / peak, 4), "traffic": traffic,
-            "peak_source": f"{peak_kind} hbm_gbs", "attention_ms": round(attn_ms, 5),
+            "peak_source": f"{pk['kind']} hbm_gbs", "attention_ms": round(attn_ms, 5),
             "algorithmic_bytes": by["attention"],
             "nominal_peak": NOMINAL_HBM_GBS,
             "frac_of_nominal": round(attn_gbs / NOMINAL_HBM_GBS, 4),
@@ -450,17 +617,24 @@ def run_native(args):
             "frac_of_read_probe": round(attn_gbs / probe, 4),
         },
         "clocks": clocks.summary(),
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": launches,
     }
     if split:
+        split["decode_rows"]["frac"] = round(split["decode_rows"]["kv_gbs"] / peak, 4)
+        split["chunks"]["frac_of_bf16_peak"] = round(split["chunks"]["tflops"] / pk["bf16"], 4)
         line["split"] = split
     if e2e:
         e2e_ms, h2d, d2h = e2e
         line["e2e"] = {"value": round(by["kv"] * world / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                       "ms_per_step": round(e2e_ms, 5)}
+                       "ms_per_step": round(e2e_ms, 5),
+                       "transfers": "one packed pinned H2D + one D2H per step, on a second "
+                                    "stream, double buffered"}
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(W, budget_s=12.0)
+    # the other reference workloads, each on the same contract (not in `value`)
+    if world == 1 and plain and not args.no_sub and args.workload == DEFAULT_WORKLOAD:
+        line["configs"] = [sub_record(torch, pa, c, dev, args, pk) for c in SUB_WORKLOADS]
     print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

@@ -51,14 +51,46 @@ def bits_to_f32(bits: np.ndarray, dtype: int) -> np.ndarray:
     raise ValueError(dtype)
 
 
+def _round_into(out: np.ndarray, x: np.ndarray, dtype: int) -> None:
+    """out[:] = x rounded to the 16-bit format (nearest even), in place on x."""
+    if dtype == BF16:
+        u = x.view(np.uint32)
+        t = u >> np.uint32(16)
+        t &= np.uint32(1)
+        t += np.uint32(0x7FFF)
+        t += u
+        t >>= np.uint32(16)
+        out[:] = t
+    else:
+        out[:] = x.astype(np.float16).view(np.uint16)
+
+
+_POOL = None
+
+
+def _pool():
+    global _POOL
+    if _POOL is None:
+        import concurrent.futures
+        import os
+        _POOL = concurrent.futures.ThreadPoolExecutor(max(1, min(8, (os.cpu_count() or 1))))
+    return _POOL
+
+
 def randn_bits(rng: np.random.Generator, shape, dtype: int) -> np.ndarray:
-    """N(0,1) samples rounded to a 16-bit float format, drawn in chunks."""
+    """N(0,1) samples rounded to a 16-bit float format, drawn in chunks.
+
+    The draws are sequential (one stream from ``rng``); the rounding of each
+    chunk runs on a worker thread while the next chunk is drawn."""
     n = int(np.prod(shape))
     out = np.empty(n, dtype=np.uint16)
-    conv = f32_to_bf16_bits if dtype == BF16 else f32_to_f16_bits
+    jobs = []
     for s in range(0, n, _CHUNK):
         e = min(n, s + _CHUNK)
-        out[s:e] = conv(rng.standard_normal(e - s, dtype=np.float32))
+        x = rng.standard_normal(e - s, dtype=np.float32)
+        jobs.append(_pool().submit(_round_into, out[s:e], x, dtype))
+    for j in jobs:
+        j.result()
     return out.reshape(shape)
 
 
