@@ -136,7 +136,10 @@ size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t head
  * block_tables : device int32 [batch][max_blocks_per_seq].
  * context_lens : device int32 [batch], each in [0, max_context_len].
  * max_context_len: host upper bound of context_lens, used to size the grid
- *                and the workspace without reading device memory.
+ *                and the workspace without reading device memory.  A row
+ *                whose context_lens entry exceeds it is cut to its first
+ *                max_context_len keys and reported in the device error word
+ *                (PA_ERR_OUT_OF_RANGE from pa_device_error).
  * partition_size: tokens per split-K partition (a multiple of 64, or 0 for
  *                an automatic choice).  Sequences longer than one partition
  *                are split; partial results (running max, sum and
@@ -179,10 +182,24 @@ pa_status pa_decode_ex(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_
                        size_t workspace_bytes, void* stream);
 
 /*
- * Bytes of workspace pa_varlen needs for these sizes.
+ * Bytes of workspace pa_varlen needs for these sizes, whichever kernels the
+ * call ends up using (the worst case over both paths described below).
  */
 size_t pa_varlen_workspace_size(int32_t num_seqs, int32_t total_q, int32_t num_q_heads,
                                 int32_t head_dim, int32_t max_context_len);
+
+/*
+ * Infrastructure, not a step of the method: the workspace pa_varlen /
+ * pa_varlen_ex need for these sizes and types, no more.  When the call's
+ * prefill chunks run on the tensor-core chunk kernel (see pa_varlen) only
+ * the q_len 1 requests use split-K partials, one work row per request, so
+ * the partials are sized for num_seqs rows instead of total_q.  The figure
+ * assumes an out pointer that is 16-byte aligned; a call whose out is not
+ * needs pa_varlen_workspace_size bytes.  Returns 0 for invalid sizes.
+ */
+size_t pa_varlen_workspace_size_ex(int32_t num_seqs, int32_t total_q, int32_t num_q_heads,
+                                   int32_t num_kv_heads, int32_t head_dim, int32_t max_q_len,
+                                   int32_t max_context_len, pa_dtype q_dtype, pa_dtype kv_dtype);
 
 /*
  * Packed mixed prefill/decode attention ("推理优化与服务：从 PagedAttention 到
@@ -196,18 +213,22 @@ size_t pa_varlen_workspace_size(int32_t num_seqs, int32_t total_q, int32_t num_q
  * (causal mask aligned to the bottom right).  Rows with no visible key yield
  * zeros.  q_len 1 rows are decode rows; longer ones are prefill chunks.
  * Chunks run on the tensor-core chunk kernel when the pool is bf16/f16 with
- * head_dim 128, q has the pool's type, the GQA group is 1, 2, 4 or 8 and out
- * is 16-byte aligned; otherwise every row runs on the decode kernel.  Either
- * way the result is the same attention.
+ * head_dim 64, 128 or 256, q has the pool's type, the GQA group is a power
+ * of two up to 128 and out is 16-byte aligned; otherwise every row runs on
+ * the decode kernel.  Either way the result is the same attention.
  *
  * out, q       : device [total_q][num_q_heads][head_dim].
  * cu_seqlens_q : device int32 [num_seqs + 1], non-decreasing, cu[0] = 0,
  *                cu[num_seqs] = total_q.
  * seqlens_k    : device int32 [num_seqs], kv_len_r >= q_len_r.
- * max_q_len, max_context_len: host upper bounds of q_len_r and kv_len_r.
+ * max_q_len, max_context_len: host upper bounds of q_len_r and kv_len_r (a
+ *                request whose kv_len_r exceeds max_context_len is cut there
+ *                and reported in the device error word, as for pa_decode).
  * block_tables : device int32 [num_seqs][max_blocks_per_seq].
  * workspace    : device scratch of at least pa_varlen_workspace_size(...)
- *                bytes, 256-byte aligned.
+ *                bytes (or pa_varlen_workspace_size_ex(...) for these exact
+ *                types), 256-byte aligned; PA_ERR_WORKSPACE if smaller than
+ *                what the path the call takes needs.
  */
 pa_status pa_varlen(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dtype,
                     int32_t total_q, int32_t num_seqs, int32_t num_q_heads,
@@ -235,9 +256,12 @@ pa_status pa_varlen(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dty
  * Arguments and results are those of pa_decode minus the workspace.  Sizes
  * whose partials need more than PA_DECODE_STATIC_SCRATCH_BYTES (see
  * pa_decode_workspace_size) return PA_ERR_WORKSPACE without launching.
- * The first call on each device, made with that device current, looks up
- * the array's device address (cudaGetSymbolAddress); make that first call
- * before any stream capture.  All calls on one device share the array and
+ * The first call in each CUDA context (normally once per device), made with
+ * that device current, looks up the array's device address
+ * (cudaGetSymbolAddress) and keeps it for that context; make that first call
+ * before any stream capture.  A failed look-up returns PA_ERR_CUDA and is not
+ * kept (the next call tries again); after a device reset the new context
+ * looks the address up afresh.  All calls on one device share the array and
  * leave their partials in it: calls that overlap on the GPU (other streams,
  * other host threads) race and must be serialised by the caller.
  */
@@ -311,9 +335,23 @@ pa_status pa_varlen_ex(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_
 pa_status pa_hbm_read_probe(const void* buf, int64_t bytes, void* sink, void* stream);
 
 /*
+ * Self-test of the failure path, not part of the method (the pages have no
+ * counterpart): every wait inside this library's kernels is bounded, and a
+ * wait that runs out records PA_ERR_TIMEOUT in the device error word and lets
+ * its kernel return instead of hanging.  This call enqueues one small kernel
+ * that waits, with a short limit (a few thousand polls), on a barrier that
+ * nothing completes, so that the next pa_device_error returns
+ * PA_ERR_TIMEOUT.  The CUDA context stays usable.  Asynchronous on `stream`;
+ * PA_ERR_CUDA if the launch fails.
+ */
+pa_status pa_selftest_wait_timeout(void* stream);
+
+/*
  * Read and clear the device error word that kernels set when they skip an
- * out-of-range block id or slot (PA_ERR_OUT_OF_RANGE) or give up a bounded
- * wait (PA_ERR_TIMEOUT).  Synchronises `stream` first.  Returns PA_OK when no
+ * out-of-range block id or slot, or cut a row whose context_lens / seqlens_k
+ * entry exceeds the max_context_len it was promised (PA_ERR_OUT_OF_RANGE; the
+ * row's attention then covers its first max_context_len keys only), or give
+ * up a bounded wait (PA_ERR_TIMEOUT).  Synchronises `stream` first.  Returns PA_OK when no
  * kernel reported anything since the last call.
  */
 pa_status pa_device_error(void* stream);

@@ -11,6 +11,9 @@
 #include <cstdlib>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
+#include <utility>
+#include <vector>
 
 namespace pa {
 
@@ -58,6 +61,63 @@ EncodeTiledFn encode_fn() {
     return nullptr;
   }();
   return fn;
+}
+
+template <class F>
+F driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    return reinterpret_cast<F>(p);
+  return nullptr;
+}
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Encoded pool / query tensor maps, keyed by everything the encoding reads
+// (base address, element type, extents, box): a hit returns the very bytes a
+// fresh encode would.  A small round-robin table shared by all host threads.
+struct MapKey {
+  const void* base;
+  int kind;            // 0: pool (esz in `a`), 1: q
+  int64_t a, b, c, d, e;
+  bool operator==(const MapKey& o) const {
+    return base == o.base && kind == o.kind && a == o.a && b == o.b && c == o.c && d == o.d &&
+           e == o.e;
+  }
+};
+constexpr int kMapCacheSize = 32;
+struct MapCache {
+  std::mutex mu;
+  MapKey key[kMapCacheSize];
+  CUtensorMap map[kMapCacheSize];
+  bool used[kMapCacheSize] = {};
+  int next = 0;
+};
+MapCache& map_cache() {
+  static MapCache c;
+  return c;
+}
+bool map_lookup(const MapKey& k, CUtensorMap* out) {
+  MapCache& c = map_cache();
+  std::lock_guard<std::mutex> g(c.mu);
+  for (int i = 0; i < kMapCacheSize; ++i)
+    if (c.used[i] && c.key[i] == k) {
+      *out = c.map[i];
+      return true;
+    }
+  return false;
+}
+void map_store(const MapKey& k, const CUtensorMap& m) {
+  MapCache& c = map_cache();
+  std::lock_guard<std::mutex> g(c.mu);
+  const int i = c.next;
+  c.next = (c.next + 1) % kMapCacheSize;
+  c.key[i] = k;
+  c.map[i] = m;
+  c.used[i] = true;
 }
 
 // With PA_DEBUG set in the environment, CUDA failures are described on stderr
@@ -109,26 +169,70 @@ DecodeWorkspace decode_workspace_layout(int64_t rows, int32_t num_q_heads, int32
   return w;
 }
 
+uint64_t current_context_id() {
+  static const CtxGetCurrentFn get_cur = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  if (!get_cur || !get_id) return 0;
+  CUcontext c = nullptr;
+  if (get_cur(&c) != CUDA_SUCCESS || !c) {
+    // nothing current yet: the runtime makes the device's primary context
+    // current when asked to use the device
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess) return 0;
+    if (get_cur(&c) != CUDA_SUCCESS || !c) return 0;
+  }
+  unsigned long long id = 0;
+  if (get_id(c, &id) != CUDA_SUCCESS) return 0;
+  return static_cast<uint64_t>(id) + 1;   // 0 stays "unknown"
+}
+
+cudaError_t ensure_smem_attribute(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static std::vector<std::pair<uint64_t, const void*>> done;
+  const uint64_t ctx = current_context_id();
+  if (ctx) {
+    std::lock_guard<std::mutex> g(mu);
+    for (const auto& d : done)
+      if (d.first == ctx && d.second == kernel) return cudaSuccess;
+  }
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && ctx) {
+    std::lock_guard<std::mutex> g(mu);
+    done.emplace_back(ctx, kernel);
+  }
+  return e;
+}
+
 bool make_pool_tensor_map(CUtensorMap* map, const void* base, int kv_dtype, int64_t rows,
                           int32_t head_dim, int32_t box_rows) {
+  const int esz = (kv_dtype == PA_FP8_E4M3) ? 1 : 2;
+  const MapKey key{base, 0, esz, rows, head_dim, box_rows, 0};
+  if (map_lookup(key, map)) return true;
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  const int esz = (kv_dtype == PA_FP8_E4M3) ? 1 : 2;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(head_dim) * esz};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esz), static_cast<cuuint32_t>(box_rows)};
+  // rows of 128 bytes or more: 128-byte boxes, 128-byte swizzle; narrower rows
+  // (E4M3 at head_dim 64) as one unswizzled box per row
+  const bool narrow = static_cast<int64_t>(head_dim) * esz < 128;
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(narrow ? head_dim : 128 / esz),
+                       static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(map, esz == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16,
                    2, const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   narrow ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS && std::getenv("PA_DEBUG"))
     std::fprintf(stderr, "libpa: pool tensor map: CUresult %d\n", static_cast<int>(r));
+  if (r == CUDA_SUCCESS) map_store(key, *map);
   return r == CUDA_SUCCESS;
 }
 
 bool make_q_tensor_map(CUtensorMap* map, const void* q, int64_t total_q, int32_t num_q_heads,
                        int32_t head_dim, int32_t group, int32_t rows) {
+  const MapKey key{q, 1, total_q, num_q_heads, head_dim, group, rows};
+  if (map_lookup(key, map)) return true;
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(num_q_heads),
@@ -142,6 +246,7 @@ bool make_q_tensor_map(CUtensorMap* map, const void* q, int64_t total_q, int32_t
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS && std::getenv("PA_DEBUG"))
     std::fprintf(stderr, "libpa: q tensor map: CUresult %d\n", static_cast<int>(r));
+  if (r == CUDA_SUCCESS) map_store(key, *map);
   return r == CUDA_SUCCESS;
 }
 
@@ -200,25 +305,51 @@ size_t pa_decode_workspace_size(int32_t batch, int32_t num_q_heads, int32_t head
 }
 
 // Varlen workspace: [row_seq | row_len] int32 [total_q] each, the prefill
-// work list (int2 [capacity] + a count), then the split-K partials for
-// max(total_q, num_seqs) rows.
-static int64_t varlen_rows(int32_t num_seqs, int32_t total_q) {
-  return total_q > num_seqs ? total_q : num_seqs;
+// work list (int2 [capacity] + a count and a unit counter), then the split-K
+// partials.  With the chunk path the decode kernel sees one work row per
+// request (num_seqs rows); without it one per packed query row (total_q).
+static int64_t varlen_head_bytes(int32_t num_seqs, int32_t total_q) {
+  const int64_t maps = 2 * align_up(static_cast<int64_t>(total_q) * 4, kAlign);
+  const int64_t items =
+      align_up(static_cast<int64_t>(prefill_item_capacity(num_seqs, total_q)) * 8, kAlign) +
+      kAlign;
+  return maps + items;
+}
+
+static int64_t varlen_partials(int64_t rows, int32_t num_q_heads, int32_t head_dim,
+                               int32_t max_context_len) {
+  if (max_context_len <= 0) return 0;
+  const int32_t ps = auto_partition(rows, num_q_heads, max_context_len);
+  const int32_t parts = static_cast<int32_t>(cdiv(max_context_len, ps));
+  return static_cast<int64_t>(decode_workspace_layout(rows, num_q_heads, head_dim, parts).total);
 }
 
 size_t pa_varlen_workspace_size(int32_t num_seqs, int32_t total_q, int32_t num_q_heads,
                                 int32_t head_dim, int32_t max_context_len) {
   if (num_seqs <= 0 || total_q <= 0 || num_q_heads <= 0 || head_dim <= 0) return 0;
-  const int64_t maps = 2 * align_up(static_cast<int64_t>(total_q) * 4, kAlign);
-  const int64_t items =
-      align_up(static_cast<int64_t>(prefill_item_capacity(num_seqs, total_q)) * 8, kAlign) +
-      kAlign;
-  if (max_context_len <= 0) return static_cast<size_t>(maps + items);
-  const int64_t rows = varlen_rows(num_seqs, total_q);
-  const int32_t ps = auto_partition(rows, num_q_heads, max_context_len);
-  const int32_t parts = static_cast<int32_t>(cdiv(max_context_len, ps));
-  return static_cast<size_t>(maps + items) +
-         decode_workspace_layout(rows, num_q_heads, head_dim, parts).total;
+  const int64_t a = varlen_partials(total_q, num_q_heads, head_dim, max_context_len);
+  const int64_t b = varlen_partials(num_seqs, num_q_heads, head_dim, max_context_len);
+  return static_cast<size_t>(varlen_head_bytes(num_seqs, total_q) + (a > b ? a : b));
+}
+
+// Whether pa_varlen runs the q_len >= 2 requests on the chunk kernel.
+static bool varlen_chunk_path(int32_t max_q_len, pa_dtype q_dtype, pa_dtype kv_dtype,
+                              int32_t head_dim, int32_t group, const void* out) {
+  return max_q_len >= 2 && (out == nullptr || aligned(out, 16)) &&
+         prefill_supported(q_dtype, kv_dtype, head_dim, group);
+}
+
+size_t pa_varlen_workspace_size_ex(int32_t num_seqs, int32_t total_q, int32_t num_q_heads,
+                                   int32_t num_kv_heads, int32_t head_dim, int32_t max_q_len,
+                                   int32_t max_context_len, pa_dtype q_dtype, pa_dtype kv_dtype) {
+  if (num_seqs <= 0 || total_q <= 0 || num_q_heads <= 0 || head_dim <= 0 || num_kv_heads <= 0 ||
+      num_q_heads % num_kv_heads != 0)
+    return 0;
+  const bool chunks = varlen_chunk_path(max_q_len, q_dtype, kv_dtype, head_dim,
+                                        num_q_heads / num_kv_heads, nullptr);
+  return static_cast<size_t>(
+      varlen_head_bytes(num_seqs, total_q) +
+      varlen_partials(chunks ? num_seqs : total_q, num_q_heads, head_dim, max_context_len));
 }
 
 static pa_status check_attention(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_dtype,
@@ -286,6 +417,7 @@ static void fill_common(AttnArgs& a, void* out, pa_dtype out_dtype, const void* 
   a.num_kv_heads = cache->num_kv_heads;
   a.head_dim = cache->head_dim;
   a.group = num_q_heads / cache->num_kv_heads;
+  a.head_chunks = a.group > 8 ? (a.group + 7) / 8 : 1;
   a.num_blocks = cache->num_blocks;
   a.block_size = cache->block_size;
   a.block_tables = block_tables;
@@ -376,8 +508,13 @@ pa_status pa_varlen_ex(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_
   if (max_q_len > max_context_len) return PA_ERR_INVALID_ARG;
   if (total_q == 0) return PA_OK;
   if (num_seqs == 0) return PA_ERR_INVALID_ARG;
-  const size_t need = pa_varlen_workspace_size(num_seqs, total_q, num_q_heads, cache->head_dim,
-                                               max_context_len);
+  const int32_t group = num_q_heads / cache->num_kv_heads;
+  const bool chunks = varlen_chunk_path(max_q_len, q_dtype, cache->kv_dtype, cache->head_dim,
+                                        group, out);
+  const int64_t rows = chunks ? num_seqs : total_q;
+  const size_t need = static_cast<size_t>(
+      varlen_head_bytes(num_seqs, total_q) +
+      varlen_partials(rows, num_q_heads, cache->head_dim, max_context_len));
   if (!workspace || workspace_bytes < need) return PA_ERR_WORKSPACE;
   if (!aligned(workspace, 256)) return PA_ERR_INVALID_ARG;
   auto* b = static_cast<uint8_t*>(workspace);
@@ -391,9 +528,6 @@ pa_status pa_varlen_ex(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_
   uint8_t* partials = b + 2 * map_bytes + item_bytes;
   const size_t head = static_cast<size_t>(2 * map_bytes + item_bytes);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int32_t group = num_q_heads / cache->num_kv_heads;
-  const bool chunks = max_q_len >= 2 && aligned(out, 16) &&
-                      prefill_supported(q_dtype, cache->kv_dtype, cache->head_dim, group);
   AttnArgs a;
   fill_common(a, out, out_dtype, q, q_dtype, num_q_heads, k_cache, v_cache, cache, block_tables,
               max_blocks_per_seq, scale);
@@ -420,7 +554,7 @@ pa_status pa_varlen_ex(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_
     p.max_context_len = max_context_len;
     p.pf_items = items;
     p.pf_count = item_count;
-    cudaError_t fe = launch_paged_prefill(p, kmap, vmap, qmap, capacity, s);
+    cudaError_t fe = launch_paged_prefill(p, kmap, vmap, qmap, capacity, item_count + 1, s);
     if (fe != cudaSuccess) return cuda_fail(fe, "prefill launch");
     a.rows = num_seqs;
     a.varlen_requests = 1;
@@ -432,9 +566,9 @@ pa_status pa_varlen_ex(void* out, pa_dtype out_dtype, const void* q, pa_dtype q_
     a.row_seq = row_seq;
     a.row_len = row_len;
   }
-  const int32_t ps = auto_partition(varlen_rows(num_seqs, total_q), num_q_heads, max_context_len);
-  const int32_t parts = static_cast<int32_t>(cdiv(max_context_len > 0 ? max_context_len : 1, ps));
-  const size_t part_need = decode_workspace_layout(a.rows, num_q_heads, cache->head_dim, parts).total;
+  const int32_t ps = auto_partition(rows, num_q_heads, max_context_len > 0 ? max_context_len : 1);
+  const size_t part_need =
+      static_cast<size_t>(varlen_partials(rows, num_q_heads, cache->head_dim, max_context_len));
   return run_attention(a, cache, max_context_len, ps, reinterpret_cast<float*>(partials),
                        workspace_bytes - head, part_need, s);
 }
@@ -524,6 +658,11 @@ pa_status pa_hbm_read_probe(const void* buf, int64_t bytes, void* sink, void* st
   cudaError_t e = launch_hbm_read_probe(buf, bytes, static_cast<uint32_t*>(sink),
                                         static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PA_OK : cuda_fail(e, "hbm_read_probe launch");
+}
+
+pa_status pa_selftest_wait_timeout(void* stream) {
+  cudaError_t e = launch_wait_timeout_selftest(static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : cuda_fail(e, "wait-timeout self-test launch");
 }
 
 pa_status pa_device_error(void* stream) {

@@ -141,6 +141,20 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
   return d;
 }
 
+// try_wait with a suspend-time hint: the thread may sleep until the phase
+// completes (or `ns` nanoseconds pass) instead of polling.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n"
+      " mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Pack two floats, `lo` into the low half: round to nearest even.
 template <bool IS_BF16>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {

@@ -9,7 +9,13 @@
 namespace pa {
 
 // Device error word codes (the first one reported wins until the host clears it).
-enum : unsigned { kErrNone = 0, kErrBlockRange = 1, kErrSlotRange = 2, kErrTimeout = 3 };
+enum : unsigned {
+  kErrNone = 0,
+  kErrBlockRange = 1,   // a block id read from a table lies outside the pool
+  kErrSlotRange = 2,    // a slot lies outside the pool
+  kErrTimeout = 3,      // a bounded wait gave up
+  kErrLenRange = 4      // a row's key count exceeds max_context_len (cut there)
+};
 
 // Everything one attention launch needs; plain pointers and sizes.
 struct AttnArgs {
@@ -18,6 +24,7 @@ struct AttnArgs {
   int out_dtype, q_dtype, kv_dtype;
   int32_t rows;                 // query rows (sequences for decode, total_q for varlen)
   int32_t num_q_heads, num_kv_heads, head_dim, group;
+  int32_t head_chunks;          // decode: query heads of a group taken 8 at a time (>= 1)
   int32_t num_blocks, block_size;
   const int32_t* block_tables;  // [num_seqs][max_blocks_per_seq]
   int32_t max_blocks_per_seq;
@@ -71,11 +78,13 @@ cudaError_t launch_varlen_prep(int32_t total_q, int32_t num_seqs, const int32_t*
 bool prefill_supported(int q_dtype, int kv_dtype, int32_t head_dim, int32_t group);
 int prefill_query_tile(int32_t group);
 int32_t prefill_item_capacity(int32_t num_seqs, int32_t total_q);
-// Builds the (request, query tile) list in a.pf_items / a.pf_count, then runs
-// the tensor-core prefill over it (grid = capacity x KV heads).
+int prefill_tiles_per_item(int32_t head_dim);
+// Builds the (request, pair of query tiles) list in a.pf_items / a.pf_count
+// (heaviest first) and resets *unit_counter, then runs the persistent
+// tensor-core prefill over it (one CTA per SM taking units through the counter).
 cudaError_t launch_paged_prefill(const AttnArgs& a, const CUtensorMap& kmap,
                                  const CUtensorMap& vmap, const CUtensorMap& qmap,
-                                 int32_t capacity, cudaStream_t stream);
+                                 int32_t capacity, int32_t* unit_counter, cudaStream_t stream);
 
 // 3-D tensor map over q [total_q][Hq][D] (16-bit), box {64, group, rows}.
 bool make_q_tensor_map(CUtensorMap* map, const void* q, int64_t total_q, int32_t num_q_heads,
@@ -109,5 +118,19 @@ cudaError_t launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* mapp
                                cudaStream_t stream);
 
 unsigned int read_and_clear_error_word(cudaStream_t stream, cudaError_t* err);
+
+// One CTA that waits, with a short poll limit, on an mbarrier nothing
+// completes, then records kErrTimeout (the bounded-wait path, exercised).
+cudaError_t launch_wait_timeout_selftest(cudaStream_t stream);
+
+// Identity of the CUDA context current on the calling thread (cuCtxGetId:
+// unique for the life of the process, so a context destroyed by a device
+// reset and its successor differ); 0 when it cannot be had.
+uint64_t current_context_id();
+
+// cudaFuncSetAttribute(kernel, MaxDynamicSharedMemorySize, bytes), done once
+// per (context, kernel): the setting belongs to the function in the current
+// context and outlives the call.
+cudaError_t ensure_smem_attribute(const void* kernel, int bytes);
 
 }  // namespace pa

@@ -39,6 +39,7 @@ constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr int kBlockTokens = 16;
 constexpr int kMaxPartitionBlocks = 128;  // partition_size <= 1024 tokens, blocks >= 8 tokens
+constexpr int kMaxGroup = 128;            // query heads per KV head
 constexpr float kLog2e = 1.4426950408889634f;
 
 enum { KV_F16 = 0, KV_BF16 = 1, KV_FP8 = 2 };
@@ -47,11 +48,16 @@ template <int KVT, int D>
 struct Geo {
   static constexpr int kElemBytes = (KVT == KV_FP8) ? 1 : 2;
   static constexpr int kRowBytes = D * kElemBytes;
-  static constexpr int kBoxBytes = kBlockTokens * 128;   // 16 rows x 128 bytes
-  static constexpr int kBoxes = kRowBytes / 128;
-  static constexpr int kBoxElems = 128 / kElemBytes;
+  // rows of 128 bytes or more travel as 128-byte boxes with the 128-byte
+  // swizzle; narrower rows (E4M3 at head_dim 64: 64 bytes) as one unswizzled box
+  static constexpr bool kNarrow = kRowBytes < 128;
+  static constexpr int kPitch = kNarrow ? kRowBytes : 128;   // bytes per box row
+  static constexpr int kBoxBytes = kBlockTokens * kPitch;
+  static constexpr int kBoxes = kRowBytes / kPitch;
+  static constexpr int kBoxElems = kPitch / kElemBytes;
   static constexpr int kTileBytes = kBoxes * kBoxBytes;
-  static_assert(kRowBytes % 128 == 0, "rows must be whole 128-byte boxes");
+  static_assert(kRowBytes % kPitch == 0, "rows must be whole boxes");
+  static_assert(!kNarrow || KVT == KV_FP8, "narrow rows only for E4M3 pools");
 };
 
 template <int KVT, int D, int GT, int NSTAGE>
@@ -119,8 +125,12 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
   const int r = lane >> 2;
   const int c = lane & 3;
 
-  // ---- work item: (row, kv head, partition)
+  // ---- work item: (row, kv head, partition, chunk of at most 8 query heads);
+  // the chunks of one (row, head, partition) are adjacent blocks, so a group
+  // larger than 8 reads each K/V tile from HBM once and from L2 after that
   int64_t bid = blockIdx.x;
+  const int chunk = static_cast<int>(bid % a.head_chunks);
+  bid /= a.head_chunks;
   const int part = static_cast<int>(bid % a.max_parts);
   bid /= a.max_parts;
   const int h = static_cast<int>(bid % a.num_kv_heads);
@@ -128,9 +138,12 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
   int seq, L, qrow;
   resolve_row(a, row, seq, L, qrow);
   if (L < 0) return;               // a varlen row owned by the prefill kernel
-  L = min(L, a.max_context_len);   // a row longer than the promised bound is cut there
-  const int group = a.group;
-  const int hq0 = h * group;
+  if (L > a.max_context_len) {     // a row longer than the promised bound is cut there
+    if (part == 0 && h == 0 && threadIdx.x == 0) report_error(kErrLenRange);
+    L = a.max_context_len;
+  }
+  const int group = min(a.group - chunk * GT, GT);   // query heads of this chunk
+  const int hq0 = h * a.group + chunk * GT;
   const int Hq = a.num_q_heads;
   if (L <= 0) {
     if (part == 0)
@@ -187,8 +200,10 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
       tma_load_2d(kt + b * G::kBoxBytes, &kmap, b * G::kBoxElems, y0, bar, policy);
       tma_load_2d(kt + kTB + b * G::kBoxBytes, &vmap, b * G::kBoxElems, y0, bar, policy);
       if (y1 >= 0) {          // 8-token blocks: rows 8..15 of the tile from the next block
-        tma_load_2d(kt + b * G::kBoxBytes + 1024, &kmap, b * G::kBoxElems, y1, bar, policy);
-        tma_load_2d(kt + kTB + b * G::kBoxBytes + 1024, &vmap, b * G::kBoxElems, y1, bar, policy);
+        tma_load_2d(kt + b * G::kBoxBytes + 8 * G::kPitch, &kmap, b * G::kBoxElems, y1, bar,
+                    policy);
+        tma_load_2d(kt + kTB + b * G::kBoxBytes + 8 * G::kPitch, &vmap, b * G::kBoxElems, y1,
+                    bar, policy);
       }
     }
   };
@@ -215,7 +230,7 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
     } else {
 #pragma unroll
       for (int p = 0; p < D / 64; ++p) {
-        const int base = (p >> 1) * 128 + 16 * (2 * c + (p & 1));
+        const int base = G::kNarrow ? 16 * c : (p >> 1) * 128 + 16 * (2 * c + (p & 1));
         uint4 w0 = make_uint4(0, 0, 0, 0), w1 = w0;
         if (live) {
           w0 = *reinterpret_cast<const uint4*>(qptr + base);
@@ -289,12 +304,13 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
       // slots); P is 0 there but 0 * NaN is NaN, so clear those V rows.
       uint8_t* vz = wt + s * 2 * kTB + kTB;
       const int dead_rows = kBlockTokens - valid;
-      for (int idx = lane; idx < dead_rows * G::kBoxes * 8; idx += 32) {
-        const int chunk = idx & 7;
-        const int rb = idx >> 3;
+      constexpr int kChunks = G::kPitch / 16;               // 16-byte chunks per box row
+      for (int idx = lane; idx < dead_rows * G::kBoxes * kChunks; idx += 32) {
+        const int chunk = idx % kChunks;
+        const int rb = idx / kChunks;
         const int box = rb / dead_rows;
         const int rw = valid + (rb - box * dead_rows);
-        *reinterpret_cast<uint4*>(vz + box * G::kBoxBytes + rw * 128 + chunk * 16) =
+        *reinterpret_cast<uint4*>(vz + box * G::kBoxBytes + rw * G::kPitch + chunk * 16) =
             make_uint4(0, 0, 0, 0);
       }
       fence_proxy_async_smem();   // order these writes before the next TMA into the stage
@@ -319,8 +335,10 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
         for (int p = 0; p < D / 64; ++p) {
           const int box = p >> 1;
           const int ch = 2 * c + (p & 1);
-          const uint4 R0 = lds128(kt_s + box * G::kBoxBytes + swz(r, ch));
-          const uint4 R8 = lds128(kt_s + box * G::kBoxBytes + swz(r + 8, ch));
+          const uint4 R0 = G::kNarrow ? lds128(kt_s + r * G::kPitch + 16 * c)
+                                      : lds128(kt_s + box * G::kBoxBytes + swz(r, ch));
+          const uint4 R8 = G::kNarrow ? lds128(kt_s + (r + 8) * G::kPitch + 16 * c)
+                                      : lds128(kt_s + box * G::kBoxBytes + swz(r + 8, ch));
           const uint32_t w0[4] = {R0.x, R0.y, R0.z, R0.w};
           const uint32_t w8[4] = {R8.x, R8.y, R8.z, R8.w};
 #pragma unroll
@@ -420,6 +438,30 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
           for (int nt = 0; nt < kNT; ++nt)
             mma16816<kMmaBF16>(acc[nt][mt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
         }
+      } else if constexpr (G::kNarrow) {
+        // 64-byte rows: lane (r, c) reads 16 dims (chunk r % 4) of tokens 2c,
+        // 2c+1, 2c+8, 2c+9 and takes the 8 starting at 8 (r / 4); m-tile t
+        // row r (r + 8) is dim 16 (r % 4) + 8 (r / 4) + 2t (+ 1)
+        const int ch = r & 3, hv = r >> 2;
+        const uint4 W0 = lds128(vt_s + (2 * c) * G::kPitch + 16 * ch);
+        const uint4 W1 = lds128(vt_s + (2 * c + 1) * G::kPitch + 16 * ch);
+        const uint4 W2 = lds128(vt_s + (2 * c + 8) * G::kPitch + 16 * ch);
+        const uint4 W3 = lds128(vt_s + (2 * c + 9) * G::kPitch + 16 * ch);
+        const uint32_t x0[2] = {hv ? W0.z : W0.x, hv ? W0.w : W0.y};
+        const uint32_t x1[2] = {hv ? W1.z : W1.x, hv ? W1.w : W1.y};
+        const uint32_t x2[2] = {hv ? W2.z : W2.x, hv ? W2.w : W2.y};
+        const uint32_t x3[2] = {hv ? W3.z : W3.x, hv ? W3.w : W3.y};
+#pragma unroll
+        for (int t = 0; t < kMTiles; ++t) {
+          const uint32_t sel = (t & 1) ? 0x7362u : 0x5140u;
+          const uint32_t lo01 = __byte_perm(x0[t >> 1], x1[t >> 1], sel);
+          const uint32_t lo23 = __byte_perm(x2[t >> 1], x3[t >> 1], sel);
+          const uint32_t a0 = e4m3x2_to_f16x2(lo01), a1 = e4m3x2_to_f16x2(lo01 >> 16);
+          const uint32_t a2 = e4m3x2_to_f16x2(lo23), a3 = e4m3x2_to_f16x2(lo23 >> 16);
+#pragma unroll
+          for (int nt = 0; nt < kNT; ++nt)
+            mma16816<false>(acc[nt][t], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+        }
       } else {
 #pragma unroll
         for (int box = 0; box < G::kBoxes; ++box) {
@@ -434,6 +476,7 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
           const uint32_t x3[4] = {W3.x, W3.y, W3.z, W3.w};
 #pragma unroll
           for (int mm = 0; mm < 8; ++mm) {
+            // bytes (k of token t, k of token t+1, k+1 of t, k+1 of t+1)
             const uint32_t sel = (mm & 1) ? 0x7362u : 0x5140u;
             const uint32_t lo01 = __byte_perm(x0[mm >> 1], x1[mm >> 1], sel);
             const uint32_t lo23 = __byte_perm(x2[mm >> 1], x3[mm >> 1], sel);
@@ -499,6 +542,9 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
         if constexpr (!kFP8) {
           d0 = 16 * mt + r;
           d1 = d0 + 8;
+        } else if constexpr (G::kNarrow) {
+          d0 = 16 * (r & 3) + 8 * (r >> 2) + 2 * mt;
+          d1 = d0 + 1;
         } else {
           d0 = (mt >> 3) * 128 + 16 * r + 2 * (mt & 7);
           d1 = d0 + 1;
@@ -553,17 +599,17 @@ __global__ void __launch_bounds__(kThreads) lse_reduce_kernel(const __grid_const
   if (nparts <= 1) return;
   const int group = a.group, D = a.head_dim, Hq = a.num_q_heads;
   const int hq0 = h * group;
-  __shared__ float s_M[16], s_inv[16];
-  if (threadIdx.x < group) {
-    const int64_t base = (static_cast<int64_t>(row) * Hq + hq0 + threadIdx.x) * a.max_parts;
+  __shared__ float s_M[kMaxGroup], s_inv[kMaxGroup];
+  const float vm = (a.kv_dtype == KV_FP8) ? a.v_scale[h] : 1.f;
+  for (int g = threadIdx.x; g < group; g += blockDim.x) {
+    const int64_t base = (static_cast<int64_t>(row) * Hq + hq0 + g) * a.max_parts;
     float M = -INFINITY;
     for (int p = 0; p < nparts; ++p) M = fmaxf(M, a.ws_m[base + p]);
     const float Mu = (M == -INFINITY) ? 0.f : M;
     float lsum = 0.f;
     for (int p = 0; p < nparts; ++p) lsum += fast_exp2(a.ws_m[base + p] - Mu) * a.ws_l[base + p];
-    const float vm = (a.kv_dtype == KV_FP8) ? a.v_scale[h] : 1.f;
-    s_M[threadIdx.x] = Mu;
-    s_inv[threadIdx.x] = lsum > 0.f ? vm / lsum : 0.f;
+    s_M[g] = Mu;
+    s_inv[g] = lsum > 0.f ? vm / lsum : 0.f;
   }
   __syncthreads();
   for (int idx = threadIdx.x; idx < group * D; idx += blockDim.x) {
@@ -606,12 +652,13 @@ cudaError_t launch_typed(const AttnArgs& a, const CUtensorMap& kmap, const CUten
   constexpr int NSTAGE = 2;
   using S = Smem<KVT, D, GT, NSTAGE>;
   auto kern = paged_attn_kernel<KVT, Q_BF16, D, GT, NSTAGE>;
-  const int64_t grid = static_cast<int64_t>(a.rows) * a.num_kv_heads * a.max_parts;
+  const int64_t grid =
+      static_cast<int64_t>(a.rows) * a.num_kv_heads * a.max_parts * a.head_chunks;
+  if (grid > 0x7fffffff) return cudaErrorInvalidConfiguration;
   if (grid == 0) return cudaSuccess;
-  // the shared-memory limit is a per-device setting of the function: set it
-  // for the current device on every launch (a host-side call)
-  cudaError_t se =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kTotal);
+  // the shared-memory limit is a setting of the function in the current
+  // context: made once per context
+  cudaError_t se = ensure_smem_attribute(reinterpret_cast<const void*>(kern), S::kTotal);
   if (se != cudaSuccess) return se;
   kern<<<static_cast<unsigned>(grid), kThreads, S::kTotal, stream>>>(a, kmap, vmap);
   cudaError_t e = cudaGetLastError();
@@ -635,9 +682,7 @@ template <int KVT, bool Q_BF16>
 cudaError_t launch_dim(const AttnArgs& a, const CUtensorMap& k, const CUtensorMap& v,
                        cudaStream_t s) {
   switch (a.head_dim) {
-    case 64:
-      if constexpr (KVT != KV_FP8) return launch_group<KVT, Q_BF16, 64>(a, k, v, s);
-      break;
+    case 64: return launch_group<KVT, Q_BF16, 64>(a, k, v, s);
     case 128: return launch_group<KVT, Q_BF16, 128>(a, k, v, s);
     case 256: return launch_group<KVT, Q_BF16, 256>(a, k, v, s);
     default: break;
@@ -648,14 +693,14 @@ cudaError_t launch_dim(const AttnArgs& a, const CUtensorMap& k, const CUtensorMa
 }  // namespace
 
 bool attention_supported(int q_dtype, int kv_dtype, int32_t head_dim, int32_t group) {
-  if (group < 1 || group > 8) return false;
+  if (group < 1 || group > kMaxGroup) return false;
   if (kv_dtype == KV_F16 || kv_dtype == KV_BF16) {
     if (q_dtype != kv_dtype) return false;
     return head_dim == 64 || head_dim == 128 || head_dim == 256;
   }
   if (kv_dtype == KV_FP8) {
     if (q_dtype != KV_F16 && q_dtype != KV_BF16) return false;
-    return head_dim == 128 || head_dim == 256;
+    return head_dim == 64 || head_dim == 128 || head_dim == 256;
   }
   return false;
 }

@@ -8,137 +8,209 @@
 // kv_len keys (cached context + this chunk, already in the paged pool), row i
 // attends keys 0 .. kv_len - q_len + i through the request's block table.
 //
-// One CTA = (request, KV head, tile of 128/G query positions); the G query
-// heads of the GQA group are stacked so the Q tile is a dense 128-row operand
-// and every K/V tile is read once for the whole group.  Per 128-key tile:
-//   S = Q K^T        tcgen05.mma kind::f16, A = Q and B = K from shared memory
-//                    (128-byte swizzle, K-major), D = S in TMEM (fp32);
-//   P = softmax row  one thread per row reads its TMEM lane, writes P as
-//                    bf16/f16 hi + lo halves back over the S columns it has read;
-//   O += P V         tcgen05.mma with A = P straight from TMEM and B = V from
-//                    shared memory (MN-major), D = O in TMEM.
+// Work unit = (request, pair of query tiles, KV head).  A query tile is
+// 128/G consecutive positions x the G query heads of the GQA group, stacked
+// into a dense 128-row operand, so every K/V tile is read once for the whole
+// group and shared by both query tiles of the pair (one for head_dim 256).
+// Per 64-key tile and query tile i:
+//   S_i = Q_i K^T    tcgen05.mma kind::f16, A = Q_i and B = K from shared
+//                    memory (128-byte swizzle, K-major), D = S_i in TMEM (fp32);
+//   P_i = softmax    one thread per row reads its TMEM lane of S_i and writes
+//                    P_i (a separate TMEM region) as 16-bit hi + lo halves;
+//   O_i += P_i V     tcgen05.mma with A = P_i from TMEM and B = V from shared
+//                    memory (MN-major), D = O_i in TMEM.
 // Softmax is online in one pass: P is taken against a running row maximum
-// that is only raised (and O, l rescaled in TMEM / registers) when a tile's
-// maximum exceeds it by more than 2^8, so P <= 256 and rescaling is rare.
-// Warp roles: 8 softmax warps in two groups of four that take alternate key
-// tiles (one thread per tile row, all 128 columns); a group passes the row
-// maxima it used to the other through shared memory, so the exponentials of
-// one group overlap the TMEM loads, maxima and stores of the other.  2 TMA
-// producer warps (K and V; paged tiles gathered 16 tokens at a time), 1 warp
-// that allocates TMEM and issues the MMAs (one lane elected per instruction).
-// S/P live in three TMEM buffers: S runs up to two tiles ahead of PV.
+// that is only raised (and O_i, l rescaled) when a tile's maximum exceeds it
+// by more than 2^8, so P <= 256 and rescaling is rare.
+//
+// Warp roles: one softmax group of 4 warps per query tile (each owns its
+// tile's rows, running maximum, sum and O, so the groups never wait on each
+// other); a K and a V producer warp (paged tiles gathered 16 tokens at a time
+// by TMA through the block table); one MMA-issuing warp per query tile, which
+// issues S_i(j+1) while softmax i still works on tile j and PV_i(j) once P_i(j)
+// is written.  S_i and P_i are separate TMEM regions: S_i(j+1) can be
+// computed while PV_i(j) still reads P_i(j).
+//
+// CTAs are persistent (one per SM): each takes units from a heaviest-first
+// list through an atomic counter until the list is exhausted.
 #include "pa_device.cuh"
 #include "pa_launch.h"
 
 namespace pa {
 namespace {
 
-constexpr int kSoftmaxWarps = 8;         // two groups of four: even and odd key tiles
-constexpr int kSoftmaxThreads = kSoftmaxWarps * 32;
-constexpr int kGroupThreads = kSoftmaxThreads / 2;
-constexpr int kProducerWarps = 2;        // one streams K tiles, one V tiles
-constexpr int kProducerWarp0 = 8;
-constexpr int kMmaWarp = kProducerWarp0 + kProducerWarps;
-constexpr int kPfThreads = (kMmaWarp + 1) * 32;
-constexpr int kBN = 128;                 // keys per tile
-constexpr int kHalf = 128 * 128;         // one 64-column (128-byte) half of a 128-row tile
-constexpr int kQBytes = 2 * kHalf;
-constexpr int kTileBytes = 2 * kHalf;    // one K or V tile: 128 keys x 128 dims
-constexpr int kKStages = 3;              // K is freed as soon as S is computed
-constexpr int kVStages = 2;              // V is freed when PV has run
-constexpr int kSBufs = 3;                // S/P buffers in TMEM
-constexpr int kKOff = kQBytes;
-constexpr int kVOff = kKOff + kKStages * kTileBytes;
+constexpr int kBN = 64;                  // keys per tile
 constexpr int kTblMax = 2048;            // block-table entries cached in shared memory
-constexpr int kTblOff = kVOff + kVStages * kTileBytes;
-constexpr int kRedOff = kTblOff + kTblMax * 4;   // [2 slots][128] maxima, [2 groups][128] sums
-constexpr int kBarBase = kRedOff + 4 * 128 * 4;
+constexpr uint32_t kWaitLimit = 1u << 15;      // hinted waits of up to 50 us each: ~1.6 s
+constexpr uint32_t kWaitHintNs = 50000;
 constexpr float kRescaleGap = 8.f;       // raise the running max when exceeded by 2^8
-// barriers: Q | K full x3 | K empty x3 | V full x2 | V empty x2 | S full x3 | P full x3 |
-//           PV done x3 | O | row maxima published [2 slots][4 lane quarters]
-enum { B_Q = 0, B_KF = 1, B_KE = 4, B_VF = 7, B_VE = 9, B_SF = 11, B_PF = 14, B_PVD = 17,
-       B_O = 20, B_MX = 21, kNumBars = 29 };
-constexpr int kSmemBytes = kBarBase + kNumBars * 8 + 16 + 1024;
-constexpr uint32_t kTmemCols = 512;      // S/P buffers at columns 0, 128, 256; O at 384
-constexpr uint32_t kOCol = 384;
-constexpr uint32_t kWaitLimit = 1u << 20;
 constexpr float kLog2eF = 1.4426950408889634f;
+constexpr uint32_t kTmemCols = 512;
+
+template <int D>
+struct Cfg {
+  static constexpr int NQ = (D == 256) ? 1 : 2;            // query tiles per unit
+  static constexpr int kCB = D / 64;                       // 128-byte column blocks
+  static constexpr int kQCB = 128 * 128;                   // bytes of a query tile column block
+  static constexpr int kQBytes = kCB * kQCB;
+  static constexpr int kKVCB = kBN * 128;                  // bytes of a K/V tile column block
+  static constexpr int kKVBytes = kCB * kKVCB;
+  static constexpr int kKSt = (D == 256) ? 2 : 4;
+  static constexpr int kVSt = (D == 256) ? 2 : 4;
+  static constexpr int kSoftmaxWarps = 4 * NQ;
+  static constexpr int kKWarp = kSoftmaxWarps;             // K producer
+  static constexpr int kVWarp = kSoftmaxWarps + 1;         // V producer
+  static constexpr int kMmaWarp0 = kSoftmaxWarps + 2;      // MMA warp i issues for query tile i
+  static constexpr int kThreads = (kMmaWarp0 + NQ) * 32;
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = NQ * kQBytes;
+  static constexpr int kVOff = kKOff + kKSt * kKVBytes;
+  static constexpr int kTblOff = kVOff + kVSt * kKVBytes;
+  static constexpr int kBarOff = kTblOff + kTblMax * 4;
+  // barriers: Q full [NQ] | K full, empty [kKSt] | V full, empty [kVSt] |
+  //           S full, S free, P full, PV done [NQ] | drain [NQ] | V fixed
+  static constexpr int B_Q = 0, B_KF = NQ, B_KE = B_KF + kKSt, B_VF = B_KE + kKSt,
+                       B_VE = B_VF + kVSt, B_SF = B_VE + kVSt, B_SE = B_SF + NQ,
+                       B_PF = B_SE + NQ, B_PVD = B_PF + NQ, B_DR = B_PVD + NQ,
+                       B_VX = B_DR + NQ, kBars = B_VX + 1;
+  static constexpr int kMiscOff = kBarOff + kBars * 8;     // tmem base, abort, unit slots
+  // + alignment slack; at least 116 KiB so that two CTAs never share an SM
+  // (each allocates all 512 TMEM columns)
+  static constexpr int kSmem = (kMiscOff + 64 + 1024) > 116 * 1024 ? (kMiscOff + 64 + 1024)
+                                                                    : 116 * 1024;
+  // TMEM columns: S_i at 64 i, P_i at 128 + 64 i, O_i at 256 + D i
+  static constexpr uint32_t kSCol = 0, kPCol = 128, kOCol = 256;
+  static_assert(kOCol + NQ * D <= kTmemCols, "TMEM budget");
+  static_assert(kSmem <= 227 * 1024, "shared-memory budget");
+};
 
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
                                               volatile int* abort_flag) {
   for (uint32_t i = 0; i < kWaitLimit; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 1023) == 1023 && *abort_flag) return false;
+    if (mbar_try_wait_hint(bar, parity, kWaitHintNs)) return true;
+    if (*abort_flag) return false;
   }
   *abort_flag = 1;
   report_error(kErrTimeout);
   return false;
 }
 
-template <bool BF16, int G>
-__global__ void __launch_bounds__(kPfThreads, 1)
+// Geometry of query tile i of a unit: its rows, positions and the 64-key tiles
+// it visits (jlo .. nkv-1; none when rows <= 0).
+struct QTile {
+  int rows, pos0, last, jlo, nkv;
+  __device__ __forceinline__ bool active(int j) const { return rows > 0 && j >= jlo && j < nkv; }
+  __device__ __forceinline__ int count() const { return rows > 0 ? nkv - jlo : 0; }
+};
+
+__device__ __forceinline__ QTile qtile(int q_len, int kv_len, int tq, int qt, int window) {
+  QTile t;
+  t.rows = min(tq, q_len - qt * tq);
+  t.pos0 = kv_len - q_len + qt * tq;
+  t.last = t.pos0 + t.rows - 1;
+  if (t.rows <= 0 || t.last < 0) {
+    t.rows = 0;
+    t.jlo = t.nkv = 0;
+    return t;
+  }
+  t.nkv = t.last / kBN + 1;
+  t.jlo = window > 0 ? max(0, t.pos0 - window + 1) / kBN : 0;
+  return t;
+}
+
+// Everything every role needs to know about one unit.
+template <int NQ>
+struct Unit {
+  int r, pair, h, cu0, q_len, kv_len, tq;
+  QTile qt[NQ];
+  int j0, nu;     // key tiles j0 .. j0 + nu - 1 are loaded (the union of the tiles' ranges)
+  int last_all;   // last position any row of the unit sees
+  // the last loaded tile holds slots past kv_len (the rest of the context's
+  // last 16-key block): the V producer clears them before the PVs read it
+  bool stale;
+};
+
+template <int NQ>
+__device__ __forceinline__ Unit<NQ> make_unit(const AttnArgs& a, int idx, int tq) {
+  Unit<NQ> u;
+  const int item = idx / a.num_kv_heads;
+  u.h = idx - item * a.num_kv_heads;
+  const int2 rp = a.pf_items[item];
+  u.r = rp.x;
+  u.pair = rp.y;
+  u.tq = tq;
+  u.cu0 = a.cu_seqlens_q[u.r];
+  u.q_len = a.cu_seqlens_q[u.r + 1] - u.cu0;
+  u.kv_len = min(a.seqlens_k[u.r], a.max_context_len);
+  u.j0 = 0x7fffffff;
+  int jend = 0;
+#pragma unroll
+  for (int i = 0; i < NQ; ++i) {
+    u.qt[i] = qtile(u.q_len, u.kv_len, tq, NQ * u.pair + i, a.window);
+    if (u.qt[i].rows > 0) {
+      u.j0 = min(u.j0, u.qt[i].jlo);
+      jend = max(jend, u.qt[i].nkv);
+    }
+  }
+  u.nu = jend > 0 ? jend - u.j0 : 0;
+  if (u.nu == 0) u.j0 = 0;
+  u.last_all = -1;
+#pragma unroll
+  for (int i = 0; i < NQ; ++i)
+    if (u.qt[i].rows > 0) u.last_all = max(u.last_all, u.qt[i].last);
+  u.stale = u.nu > 0 && (u.kv_len % 16) != 0 && u.last_all >= ((u.kv_len - 1) & ~15);
+  return u;
+}
+
+template <bool BF16, int D>
+__global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
 paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUtensorMap kmap,
                      const __grid_constant__ CUtensorMap vmap,
-                     const __grid_constant__ CUtensorMap qmap) {
-  constexpr int TQ = 128 / G;             // query positions per tile
+                     const __grid_constant__ CUtensorMap qmap, int log2g, int32_t* unit_counter) {
+  using C = Cfg<D>;
+  constexpr int NQ = C::NQ;
   constexpr uint32_t kIdescS = idesc_f16(BF16, 128, kBN, false);
-  constexpr uint32_t kIdescPV = idesc_f16(BF16, 128, 128, true);
+  constexpr uint32_t kIdescPV = idesc_f16(BF16, 128, D, true);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* sQ = smem;
-  int32_t* tbl = reinterpret_cast<int32_t*>(smem + kTblOff);
-  float* red = reinterpret_cast<float*>(smem + kRedOff);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBarBase);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBarBase + kNumBars * 8);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int32_t* tbl = reinterpret_cast<int32_t*>(smem + C::kTblOff);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+  volatile int* unit_slot = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 8);  // [2]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  // ---- work item from the compact list: (request, query tile) x KV head
-  const int item = blockIdx.x / a.num_kv_heads;
-  const int h = blockIdx.x - item * a.num_kv_heads;
-  if (item >= *a.pf_count) return;
-  const int2 rq = a.pf_items[item];
-  const int r = rq.x, qt = rq.y;
-  const int cu0 = a.cu_seqlens_q[r];
-  const int q_len = a.cu_seqlens_q[r + 1] - cu0;
-  const int kv_len = min(a.seqlens_k[r], a.max_context_len);
-  const int rows_valid = min(TQ, q_len - qt * TQ);
-  const int pos0 = kv_len - q_len + qt * TQ;        // absolute position of tile row 0
-  const int last_pos = pos0 + rows_valid - 1;
-  if (rows_valid <= 0 || last_pos < 0) return;
-  const int nkv = last_pos / kBN + 1;
-  // sliding window: key tiles before the first key any row of the tile sees
-  // are skipped (tiles jlo .. nkv-1 are visited, ntile of them)
-  const int jlo = a.window > 0 ? max(0, pos0 - a.window + 1) / kBN : 0;
-  const int ntile = nkv - jlo;
-  const int n_iter = ntile;
-  const int hq0 = h * G;
+  const int G = 1 << log2g;
+  const int tq = 128 >> log2g;              // query positions per tile
+  const int total_units = *a.pf_count * a.num_kv_heads;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars[B_Q], 1);
-    for (int s = 0; s < kKStages; ++s) {
-      mbar_init(&bars[B_KF + s], 1);
-      mbar_init(&bars[B_KE + s], 1);
+    for (int i = 0; i < NQ; ++i) {
+      mbar_init(&bars[C::B_Q + i], 1);
+      mbar_init(&bars[C::B_SF + i], 1);
+      mbar_init(&bars[C::B_SE + i], 128);
+      mbar_init(&bars[C::B_PF + i], 128);
+      mbar_init(&bars[C::B_PVD + i], 1);
     }
-    for (int s = 0; s < kVStages; ++s) {
-      mbar_init(&bars[B_VF + s], 1);
-      mbar_init(&bars[B_VE + s], 1);
+    // a K or V stage is free once every MMA warp's readers of it are done
+    for (int s = 0; s < C::kKSt; ++s) {
+      mbar_init(&bars[C::B_KF + s], 1);
+      mbar_init(&bars[C::B_KE + s], NQ);
     }
-    for (int s = 0; s < kSBufs; ++s) {
-      mbar_init(&bars[B_SF + s], 1);
-      mbar_init(&bars[B_PF + s], kGroupThreads);
-      mbar_init(&bars[B_PVD + s], 1);
+    for (int s = 0; s < C::kVSt; ++s) {
+      mbar_init(&bars[C::B_VF + s], 1);
+      mbar_init(&bars[C::B_VE + s], NQ);
     }
-    mbar_init(&bars[B_O], 1);
-    for (int s = 0; s < 8; ++s) mbar_init(&bars[B_MX + s], 32);
+    for (int i = 0; i < NQ; ++i) mbar_init(&bars[C::B_DR + i], 1);
+    mbar_init(&bars[C::B_VX], 1);
     *abort_flag = 0;
+    unit_slot[0] = atomicAdd(unit_counter, 1);
     fence_barrier_init();
   }
-  if (warp == kMmaWarp) {
+  if (warp == C::kMmaWarp0) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -147,381 +219,416 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp >= kProducerWarp0 && warp < kMmaWarp) {
-    // ================================================================ TMA producers
-    // One warp streams K tiles, one V tiles.  Lane 0 waits for a free stage
-    // and arms its barrier with the tile's bytes; lanes 0-7 then each fetch
-    // one 16-key sub-tile (both 64-column halves) through the block table.
-    const int pw = warp - kProducerWarp0;
-    const bool is_v = pw == 1;
-    const int32_t* bt = a.block_tables + static_cast<int64_t>(r) * a.max_blocks_per_seq;
-    const int bs = a.block_size;
-    const int nblk = last_pos / bs + 1;               // blocks holding visible keys
-    const int ncache = min(nblk, kTblMax);
-    for (int i = pw * 32 + lane; i < ncache; i += kProducerWarps * 32) tbl[i] = __ldg(bt + i);
-    named_bar(2, kProducerWarps * 32);
-    const int oob_row = a.num_blocks * a.num_kv_heads * bs;
-    if (pw == 0 && lane == 0) {
-      prefetch_tensormap(&kmap);
-      prefetch_tensormap(&vmap);
-      mbar_arrive_expect_tx(&bars[B_Q], kQBytes);
-      tma_load_3d(sQ, &qmap, 0, hq0, cu0 + qt * TQ, &bars[B_Q]);
-      tma_load_3d(sQ + kHalf, &qmap, 64, hq0, cu0 + qt * TQ, &bars[B_Q]);
-    }
-    const uint64_t pol = l2_policy_evict_last();
-    const int nstage = is_v ? kVStages : kKStages;
-    uint64_t* full = &bars[is_v ? B_VF : B_KF];
-    uint64_t* empty = &bars[is_v ? B_VE : B_KE];
-    const CUtensorMap* map = is_v ? &vmap : &kmap;
-    uint8_t* ring = smem + (is_v ? kVOff : kKOff);
-    int issued = 0;
-    for (int u = 0; u < ntile; ++u) {
-      const int j = jlo + u;                              // key tile
-      const int st = u % nstage;
-      int go = 1;
-      if (lane == 0) {
-        go = !*abort_flag;
-        if (go && u >= nstage) go = wait_or_abort(&empty[st], (u / nstage - 1) & 1, abort_flag);
-        if (go) mbar_arrive_expect_tx(&full[st], kTileBytes);
+  // Running counts of every barrier's completed phases, kept across units by
+  // the roles that wait on them (parity = count & 1).
+  uint32_t kcnt = 0, vcnt = 0;             // K / V tiles loaded (producers) or passed (others)
+  uint32_t mq = 0, ms = 0, mp = 0, mx = 0; // MMA warp: its Q loads, S tiles, PV batches, V fixes
+  uint32_t sm_s = 0, sm_p = 0;             // softmax group: its tile's S tiles and PV batches
+
+  int k = 0;
+  for (;; ++k) {
+    const int idx = unit_slot[k & 1];
+    if (idx >= total_units || *abort_flag) break;
+    const Unit<NQ> U = make_unit<NQ>(a, idx, tq);
+    const int hq0 = U.h * G;
+
+    if (warp == C::kKWarp || warp == C::kVWarp) {
+      // ============================================================ TMA producers
+      const bool is_v = warp == C::kVWarp;
+      const int32_t* bt = a.block_tables + static_cast<int64_t>(U.r) * a.max_blocks_per_seq;
+      const int bs = a.block_size;
+      const int last_all = U.last_all;
+      const int nblk = last_all / bs + 1;
+      const int ncache = min(nblk, kTblMax);
+      for (int i = (is_v ? 32 : 0) + lane; i < ncache; i += 64) tbl[i] = __ldg(bt + i);
+      named_bar(2, 64);
+      const int oob_row = a.num_blocks * a.num_kv_heads * bs;
+      if (!is_v && lane == 0) {
+        prefetch_tensormap(&kmap);
+        prefetch_tensormap(&vmap);
+#pragma unroll
+        for (int i = 0; i < NQ; ++i) {
+          if (U.qt[i].rows <= 0) continue;
+          uint64_t* qb = &bars[C::B_Q + i];
+          mbar_arrive_expect_tx(qb, C::kQBytes);
+          uint8_t* sq = smem + C::kQOff + i * C::kQBytes;
+          const int row0 = U.cu0 + (NQ * U.pair + i) * tq;
+#pragma unroll
+          for (int cb = 0; cb < C::kCB; ++cb)
+            tma_load_3d(sq + cb * C::kQCB, &qmap, cb * 64, hq0, row0, qb);
+        }
       }
-      if (!__shfl_sync(0xffffffffu, go, 0)) break;
-      if (lane < 8) {
-        // sub-tile `lane` of key tile j: one box of 16 rows (two of 8 rows
-        // for 8-token blocks); past the visible keys the box starts past the
-        // pool and is zero filled
-        const int sti = j * 8 + lane;
-        int y0 = oob_row, y1 = bs == 8 ? oob_row : -1;
-        if (sti * 16 <= last_pos) {
-          const int32_t* src = (sti + 1) * 16 / bs + 1 < kTblMax ? tbl : bt;
-          int r0, r1;
-          if (tile_rows(src, sti, bs, nblk, a.num_blocks, a.num_kv_heads, h, oob_row, r0, r1)) {
-            y0 = r0;
-            y1 = r1;
-          } else {
-            report_error(kErrBlockRange);
+      const uint64_t pol = l2_policy_evict_last();
+      const int nst = is_v ? C::kVSt : C::kKSt;
+      uint64_t* full = &bars[is_v ? C::B_VF : C::B_KF];
+      uint64_t* empty = &bars[is_v ? C::B_VE : C::B_KE];
+      const CUtensorMap* map = is_v ? &vmap : &kmap;
+      uint8_t* ring = smem + (is_v ? C::kVOff : C::kKOff);
+      uint32_t& cnt = is_v ? vcnt : kcnt;
+      for (int u = 0; u < U.nu; ++u) {
+        const int j = U.j0 + u;
+        const uint32_t st = cnt % nst;
+        int go = 1;
+        if (lane == 0) {
+          go = !*abort_flag;
+          if (go && cnt >= static_cast<uint32_t>(nst))
+            go = wait_or_abort(&empty[st], ((cnt / nst) - 1) & 1, abort_flag);
+          if (go) mbar_arrive_expect_tx(&full[st], C::kKVBytes);
+        }
+        if (!__shfl_sync(0xffffffffu, go, 0)) break;
+        if (lane < kBN / 16) {
+          // 16-key sub-tile `lane` of key tile j; past the keys any row sees
+          // the box starts past the pool and is zero filled
+          const int sti = j * (kBN / 16) + lane;
+          int y0 = oob_row, y1 = bs == 8 ? oob_row : -1;
+          if (sti * 16 <= last_all) {
+            const int32_t* src = (sti + 1) * 16 / bs + 1 < kTblMax ? tbl : bt;
+            int r0, r1;
+            if (tile_rows(src, sti, bs, nblk, a.num_blocks, a.num_kv_heads, U.h, oob_row, r0,
+                          r1)) {
+              y0 = r0;
+              y1 = r1;
+            } else {
+              report_error(kErrBlockRange);
+            }
+          }
+          uint8_t* box = ring + st * C::kKVBytes + lane * 2048;
+#pragma unroll
+          for (int cb = 0; cb < C::kCB; ++cb) {
+            tma_load_2d(box + cb * C::kKVCB, map, cb * 64, y0, &full[st], pol);
+            if (y1 >= 0)
+              tma_load_2d(box + cb * C::kKVCB + 1024, map, cb * 64, y1, &full[st], pol);
           }
         }
-        uint8_t* box = ring + st * kTileBytes + lane * 2048;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          tma_load_2d(box + half * kHalf, map, half * 64, y0, &full[st], pol);
-          if (y1 >= 0) tma_load_2d(box + half * kHalf + 1024, map, half * 64, y1, &full[st], pol);
-        }
+        ++cnt;
       }
-      issued = u + 1;
-    }
-    // the last copies into each stage have landed before the CTA may exit
-    if (lane == 0) {
-      for (int u = issued - 1; u >= 0 && u >= issued - nstage; --u)
-        (void)mbar_wait_bounded(&full[u % nstage], (u / nstage) & 1);
-      if (pw == 0) (void)mbar_wait_bounded(&bars[B_Q], 0);
-    }
-  } else if (warp == kMmaWarp) {
-    // ================================================================ MMA issuer
-    // The whole warp runs this loop converged (every wait is taken by all
-    // lanes, and agreed on); one elected lane issues each MMA and commit.
-    auto wait_all = [&](uint64_t* bar, uint32_t parity) {
-      return __all_sync(0xffffffffu, wait_or_abort(bar, parity, abort_flag));
-    };
-    bool ok = wait_all(&bars[B_Q], 0);
-    // descriptors of the first 16-column slice of Q, K stage 0 and V stage 0;
-    // a slice or stage is an offset added to the start-address field (byte
-    // address / 16, which stays below 2^14 for any shared-memory address)
-    const uint64_t q_desc = smem_desc_sw128(smem_u32(sQ), 16, 1024);
-    const uint64_t k_desc = smem_desc_sw128(smem_u32(smem + kKOff), 16, 1024);
-    const uint64_t v_desc = smem_desc_sw128(smem_u32(smem + kVOff), kHalf, 1024);
-    int next_s = 0;
-    for (int it = 0; ok && it < n_iter; ++it) {
-      // S runs up to two tiles ahead of PV, so both softmax groups have a
-      // tile to work on; buffer reuse waits for PV(next_s - 3) only
-      while (ok && next_s < n_iter && next_s <= it + 2) {
-        const int sb = next_s % kSBufs;
-        if (next_s >= kSBufs && !(ok = wait_all(&bars[B_PVD + sb], (next_s / kSBufs - 1) & 1)))
-          break;
-        const int ks = next_s % kKStages;
-        if (!(ok = wait_all(&bars[B_KF + ks], (next_s / kKStages) & 1))) break;
-        tc_fence_after();
-        const uint64_t kd = k_desc + static_cast<uint64_t>((ks * kTileBytes) >> 4);
-        const uint32_t d = tmem + static_cast<uint32_t>(sb * 128);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kHalf + (kk & 3) * 32) >> 4);
-          tc_mma_ss_warp(d, q_desc + off, kd + off, kIdescS, kk > 0 ? 1u : 0u);
-        }
-        tc_commit_warp(&bars[B_SF + sb]);
-        tc_commit_warp(&bars[B_KE + ks]);       // S is the only reader of K
-        ++next_s;
-      }
-      if (!ok) break;
-      // O += P V once the softmax group has written P(it) (and rescaled O)
-      const int b = it % kSBufs;
-      if (!(ok = wait_all(&bars[B_PF + b], (it / kSBufs) & 1))) break;
-      const int vs = it % kVStages;
-      if (!(ok = wait_all(&bars[B_VF + vs], (it / kVStages) & 1))) break;
-      tc_fence_after();
-      const uint64_t vd = v_desc + static_cast<uint64_t>((vs * kTileBytes) >> 4);
-      const uint32_t p_base = tmem + static_cast<uint32_t>(b * 128);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        // keys 16kk .. 16kk+15: chunk kk/2 of 32 keys holds 16 hi columns
-        // then 16 lo columns, 8 columns (16 packed values) per half chunk
-        const uint32_t pc = p_base + 32 * (kk >> 1) + 8 * (kk & 1);
-        const uint64_t vk = vd + static_cast<uint64_t>((kk * 2048) >> 4);
-        tc_mma_ts_warp(tmem + kOCol, pc, vk, kIdescPV, (it == 0 && kk == 0) ? 0u : 1u);
-        tc_mma_ts_warp(tmem + kOCol, pc + 16, vk, kIdescPV, 1u);
-      }
-      tc_commit_warp(&bars[B_VE + vs]);
-      tc_commit_warp(&bars[B_PVD + b]);
-    }
-    tc_commit_warp(&bars[B_O]);              // every MMA issued above is complete
-    if (!ok) (void)wait_all(&bars[B_O], 0);
-  } else {
-    // ================================================================ softmax / epilogue
-    // Group grp (warps 4*grp ..) takes key tiles grp, grp + 2, ...; warp w's
-    // 32 threads own tile rows (= TMEM lanes) 32*(w%4).., all 128 columns.
-    const int quarter = warp & 3, grp = warp >> 2;
-    const int t = quarter * 32 + lane;         // tile row == TMEM lane
-    const int i = t / G, g = t % G;
-    const bool row_ok = i < rows_valid;
-    const int pos = pos0 + i;
-    const float c = a.scale * kLog2eF;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
-    bool ok = true;
-    // Row visibility: keys lo_row .. pos (lo_row from the sliding window);
-    // logits in the log2 domain x = s*scale*log2e + slope*log2e*(key - pos).
-    const int lo_row = a.window > 0 ? pos - a.window + 1 : 0;
-    const float slope = a.alibi ? a.alibi[hq0 + g] * kLog2eF : 0.f;
-    // without ALiBi (and with scale > 0) the max is taken on the raw scores
-    // and the scale folds into the exponent's FFMA
-    const bool direct = a.alibi == nullptr && c > 0.f;
-    const float cc = direct ? c : 1.f;
-    // a tile every row sees in full needs no mask
-    auto tile_full = [&](int j) {
-      return j * kBN + kBN - 1 <= pos0 && (a.window <= 0 || j * kBN >= last_pos - a.window + 1);
-    };
-    // 32 columns of S (column0 = k0 .. k0 + 31 of the tile) -> logits in place
-    auto logits = [&](uint32_t (&v)[32], int col0, int nlo, int nhi, bool full, float b0) {
-      if (!direct) {
-#pragma unroll
-        for (int n = 0; n < 32; ++n)
-          v[n] = __float_as_uint(
-              fmaf(__uint_as_float(v[n]), c, fmaf(slope, static_cast<float>(col0 + n), b0)));
-      }
-      if (!full) {
-#pragma unroll
-        for (int n = 0; n < 32; ++n)
-          if (col0 + n < nlo || col0 + n > nhi) v[n] = __float_as_uint(-INFINITY);
-      }
-    };
-    float* m_pub = red;                        // [slot = tile & 1][row]: maximum used
-    float l_part = 0.f;                        // this group's share of the row sum,
-    float m_l = -INFINITY;                     // relative to 2^m_l
-    for (int it = grp; ok && it < n_iter; it += 2) {
-      const int b = it % kSBufs;
-      if (!wait_or_abort(&bars[B_SF + b], (it / kSBufs) & 1, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      const int j = jlo + it;
-      const int key0 = j * kBN;
-      const bool full = tile_full(j);
-      // keys outside lo_row .. pos of this row (every key of a padding row)
-      // are masked; stale slots past kv_len always fall in a masked tile
-      const int nlo = full ? 0 : (row_ok ? lo_row - key0 : kBN);
-      const int nhi = full ? kBN - 1 : (row_ok ? pos - key0 : -1);
-      const float b0 = slope * static_cast<float>(key0 - pos);
-      const uint32_t s_col = lane_base + b * 128;
-      // ---- the row of S (128 columns) in registers, one TMEM round trip;
-      // the tile's row maximum (log2 domain) in four independent chains
-      uint32_t v[4][32];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) tmem_ld32(s_col + 32 * k, v[k]);
-      tmem_wait_ld();
-      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        logits(v[k], 32 * k, nlo, nhi, full, b0);
-#pragma unroll
-        for (int n2 = 0; n2 < 16; ++n2)
-          m4[n2 & 3] = fmax3(m4[n2 & 3], __uint_as_float(v[k][2 * n2]), __uint_as_float(v[k][2 * n2 + 1]));
-      }
-      float m_tile = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-      if (direct) m_tile *= c;                 // scale > 0: the maximum commutes with it
-      // ---- the running maximum before this tile, from the group that ran
-      // tile it - 1; raise it only when this tile exceeds it by 2^8
-      float m_prev = -INFINITY;
-      if (it > 0) {
-        const int sp = (it - 1) & 1;
-        if (!wait_or_abort(&bars[B_MX + 4 * sp + quarter], ((it - 1) >> 1) & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
-        m_prev = m_pub[sp * 128 + t];
-      }
-      const bool raise = (m_prev == -INFINITY) ? (m_tile != -INFINITY)
-                                               : (m_tile > m_prev + kRescaleGap);
-      const float m_new = raise ? m_tile : m_prev;
-      m_pub[(it & 1) * 128 + t] = m_new;
-      mbar_arrive(&bars[B_MX + 4 * (it & 1) + quarter]);
-      if (m_new != m_l) {                      // rescale this group's partial sum
-        l_part = (m_l == -INFINITY) ? 0.f : l_part * fast_exp2(m_l - m_new);
-        m_l = m_new;
-      }
-      // ---- p = 2^(x - m_new) per 32-column chunk, written back over the
-      // chunk's S columns as 16 hi then 16 lo columns of packed pairs
-      const float nmu = (m_new == -INFINITY) ? 0.f : -m_new;
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        uint32_t hi[16], lo[16];
-#pragma unroll
-        for (int n2 = 0; n2 < 16; ++n2) {
-          const float p0 = fast_exp2(fmaf(__uint_as_float(v[k][2 * n2]), cc, nmu));   // 2^-inf = 0
-          const float p1 = fast_exp2(fmaf(__uint_as_float(v[k][2 * n2 + 1]), cc, nmu));
-          ls[n2 & 3] += p0 + p1;
-          const uint32_t hw = pack2<BF16>(p0, p1);
-          hi[n2] = hw;
-          lo[n2] = pack2<BF16>(p0 - lo_half_to_float<BF16>(hw), p1 - lo_half_to_float<BF16>(hw >> 16));
-        }
-        tmem_st16(s_col + 32 * k, hi);
-        tmem_st16(s_col + 32 * k + 16, lo);
-      }
-      l_part += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-      if (it > 0 && __any_sync(0xffffffffu, raise)) {
-        // O holds PV of tiles < it: wait for PV(it - 1), then scale the rows
-        // that raised their maximum (alpha = 1 elsewhere, 0 for a row whose
-        // earlier keys were all masked)
-        const float alpha = !raise ? 1.f : (m_prev == -INFINITY ? 0.f : fast_exp2(m_prev - m_new));
-        if (!wait_or_abort(&bars[B_PVD + (it - 1) % kSBufs], ((it - 1) / kSBufs) & 1,
-                           abort_flag)) {
-          ok = false;
-        }
-        tc_fence_after();
-#pragma unroll 1
-        for (int q2 = 0; q2 < 4; ++q2) {
-          uint32_t o[32];
-          tmem_ld32(lane_base + kOCol + 32 * q2, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st32(lane_base + kOCol + 32 * q2, o);
-        }
-      }
-      // Keys of the context's partial last block that lie past kv_len hold
-      // whatever the slot held; P is 0 there but 0 * NaN is NaN: clear them.
-      const int stale0 = kv_len, stale1 = min((kv_len + 15) & ~15, key0 + kBN);
-      if (stale0 < stale1 && stale0 >= key0) {
-        const int vs = it % kVStages;
-        if (wait_or_abort(&bars[B_VF + vs], (it / kVStages) & 1, abort_flag)) {
-          uint8_t* sV = smem + kVOff + vs * kTileBytes;
-          const int nrows = stale1 - stale0;
-          for (int idx = t; idx < nrows * 16; idx += kGroupThreads) {
-            const int row = stale0 - key0 + idx / 16;
-            const int c16 = idx % 16;
-            *reinterpret_cast<uint4*>(sV + (c16 >> 3) * kHalf + row * 128 + (c16 & 7) * 16) =
+      if (is_v && U.stale && !*abort_flag) {
+        // V rows of the context's last 16-key block past kv_len hold whatever
+        // the slots held; P is 0 there but 0 * NaN is NaN: once the unit's
+        // last V tile (which holds them) has landed, clear them, then let
+        // the MMA warps at it
+        const uint32_t lt = cnt - 1;
+        const bool landed = __all_sync(
+            0xffffffffu, wait_or_abort(&full[lt % nst], (lt / nst) & 1, abort_flag));
+        if (landed) {
+          uint8_t* sv = ring + (lt % nst) * C::kKVBytes;
+          const int jl = U.j0 + U.nu - 1;
+          const int r0 = U.kv_len - jl * kBN;
+          const int r1 = ((U.kv_len + 15) & ~15) - jl * kBN;
+          for (int ix = lane; ix < (r1 - r0) * 8 * C::kCB; ix += 32) {
+            const int rr = r0 + ix / (8 * C::kCB);
+            const int rem = ix % (8 * C::kCB);
+            *reinterpret_cast<uint4*>(sv + (rem >> 3) * C::kKVCB + rr * 128 + (rem & 7) * 16) =
                 make_uint4(0, 0, 0, 0);
           }
           fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&bars[C::B_VX]);
         }
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&bars[B_PF + b]);
-    }
-    // -------- epilogue: O row / l -> out (group grp writes dims 64*grp ..)
-    named_bar(1, kSoftmaxThreads);             // every tile's maximum is published
-    const float m_fin = n_iter > 0 ? m_pub[((n_iter - 1) & 1) * 128 + t] : -INFINITY;
-    red[256 + grp * 128 + t] =
-        (m_l == -INFINITY || m_fin == -INFINITY) ? 0.f : l_part * fast_exp2(m_l - m_fin);
-    named_bar(1, kSoftmaxThreads);
-    const float l_row = red[256 + t] + red[384 + t];
-    const float inv_l = l_row > 0.f ? 1.f / l_row : 0.f;
-    const int half = grp;
-    if (ok && wait_or_abort(&bars[B_O], 0, abort_flag)) {
-      tc_fence_after();
-      uint32_t o[64];
-      tmem_ld32(lane_base + kOCol + half * 64, *reinterpret_cast<uint32_t (*)[32]>(o));
-      tmem_ld32(lane_base + kOCol + half * 64 + 32, *reinterpret_cast<uint32_t (*)[32]>(o + 32));
-      tmem_wait_ld();
-      if (row_ok) {
-        const int64_t orow =
-            (static_cast<int64_t>(cu0 + qt * TQ + i) * a.num_q_heads + hq0 + g) * 128 + half * 64;
-        if (a.out_dtype == 3) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow);
+      __syncwarp();
+    } else if (warp >= C::kMmaWarp0) {
+      // ============================================================ MMA issuers
+      // Warp kMmaWarp0 + i issues every MMA of query tile i, converged, one
+      // elected lane per instruction: S_i(j) as soon as softmax i has read
+      // S_i(j-1) and K(j) has landed, then PV_i(j-1) once P_i(j-1) is
+      // written.  Its commits track only its own MMAs, so the two query
+      // tiles never wait on each other's softmax.
+      const int i = warp - C::kMmaWarp0;
+      const QTile T = (NQ == 2 && i == 1) ? U.qt[NQ - 1] : U.qt[0];
+      auto wait_all = [&](uint64_t* bar, uint32_t parity) {
+        return __all_sync(0xffffffffu, wait_or_abort(bar, parity, abort_flag));
+      };
+      bool ok = true;
+      const uint64_t qdesc =
+          smem_desc_sw128(smem_u32(smem + C::kQOff + i * C::kQBytes), 16, 1024);
+      if (T.rows > 0) {
+        ok = wait_all(&bars[C::B_Q + i], mq & 1);
+        ++mq;
+      }
+      const uint64_t kdesc0 = smem_desc_sw128(smem_u32(smem + C::kKOff), 16, 1024);
+      const uint64_t vdesc0 = smem_desc_sw128(smem_u32(smem + C::kVOff), C::kKVCB, 1024);
+      const uint32_t d_s = tmem + C::kSCol + 64 * i;
+      const uint32_t d_o = tmem + C::kOCol + D * i;
+      const uint32_t a_p = tmem + C::kPCol + 64 * i;
+      bool first_pv = true;
+      for (int u = 0; ok && u <= U.nu; ++u) {
+        const int j = U.j0 + u;
+        if (u < U.nu) {
+          // K(j) is waited for even when this tile does not need it, so that
+          // this warp's release of the stage never runs ahead of the load
+          const uint32_t ks = kcnt % C::kKSt;
+          if (!(ok = wait_all(&bars[C::B_KF + ks], (kcnt / C::kKSt) & 1))) break;
+          if (T.active(j)) {
+            // ---- S_i(j) = Q_i K(j)^T
+            if (ms > 0 && !(ok = wait_all(&bars[C::B_SE + i], (ms - 1) & 1))) break;
+            tc_fence_after();
+            const uint64_t kd = kdesc0 + static_cast<uint64_t>((ks * C::kKVBytes) >> 4);
 #pragma unroll
-          for (int k = 0; k < 16; ++k)
-            dst[k] = make_float4(__uint_as_float(o[4 * k]) * inv_l,
-                                 __uint_as_float(o[4 * k + 1]) * inv_l,
-                                 __uint_as_float(o[4 * k + 2]) * inv_l,
-                                 __uint_as_float(o[4 * k + 3]) * inv_l);
-        } else {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + orow);
-          const bool ob = (a.out_dtype == 1);
-#pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float x0 = __uint_as_float(o[8 * k + 2 * e]) * inv_l;
-              const float x1 = __uint_as_float(o[8 * k + 2 * e + 1]) * inv_l;
-              w[e] = ob ? pack2<true>(x0, x1) : pack2<false>(x0, x1);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t qo = static_cast<uint64_t>(((kk >> 2) * C::kQCB + (kk & 3) * 32) >> 4);
+              const uint64_t ko = static_cast<uint64_t>(((kk >> 2) * C::kKVCB + (kk & 3) * 32) >> 4);
+              tc_mma_ss_warp(d_s, qdesc + qo, kd + ko, kIdescS, kk > 0 ? 1u : 0u);
             }
-            dst[k] = make_uint4(w[0], w[1], w[2], w[3]);
+            tc_commit_warp(&bars[C::B_SF + i]);
+            ++ms;
+          }
+          tc_commit_warp(&bars[C::B_KE + ks]);   // this warp's reads of K(j) are done
+          ++kcnt;
+        }
+        if (u >= 1) {
+          const uint32_t vs = vcnt % C::kVSt;
+          if (!(ok = wait_all(&bars[C::B_VF + vs], (vcnt / C::kVSt) & 1))) break;
+          if (U.stale && u == U.nu) {     // the unit's last V tile, cleared by its producer
+            if (!(ok = wait_all(&bars[C::B_VX], mx & 1))) break;
+            ++mx;
+          }
+          if (T.active(j - 1)) {
+            // ---- O_i += P_i(j-1) V(j-1)
+            if (!(ok = wait_all(&bars[C::B_PF + i], mp & 1))) break;
+            tc_fence_after();
+            const uint64_t vd = vdesc0 + static_cast<uint64_t>((vs * C::kKVBytes) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < kBN / 16; ++kk) {
+              // keys 16kk .. 16kk+15: 8 columns of hi pairs, then 8 of lo pairs
+              const uint64_t vk = vd + static_cast<uint64_t>((kk * 2048) >> 4);
+              tc_mma_ts_warp(d_o, a_p + 16 * kk, vk, kIdescPV, (first_pv && kk == 0) ? 0u : 1u);
+              tc_mma_ts_warp(d_o, a_p + 16 * kk + 8, vk, kIdescPV, 1u);
+            }
+            first_pv = false;
+            tc_commit_warp(&bars[C::B_PVD + i]);
+            ++mp;
+          }
+          tc_commit_warp(&bars[C::B_VE + vs]);   // this warp's reads of V(j-1) are done
+          ++vcnt;
+        }
+      }
+      if (!ok) *abort_flag = 1;
+    } else {
+      // ============================================================ softmax / epilogue
+      const int qi = warp >> 2;                  // query tile of this group
+      const QTile T = (NQ == 2 && qi == 1) ? U.qt[NQ - 1] : U.qt[0];
+      const int quarter = warp & 3;
+      const int t = quarter * 32 + lane;         // tile row == TMEM lane
+      const int row = t >> log2g, g = t & (G - 1);
+      const bool row_ok = row < T.rows;
+      const int pos = T.pos0 + row;
+      const uint32_t lane_base = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+      const uint32_t s_col = lane_base + C::kSCol + 64 * qi;
+      const uint32_t p_col = lane_base + C::kPCol + 64 * qi;
+      const uint32_t o_col = lane_base + C::kOCol + D * qi;
+      const float c = a.scale * kLog2eF;
+      const int lo_row = a.window > 0 ? pos - a.window + 1 : 0;
+      const float slope = a.alibi ? a.alibi[hq0 + g] * kLog2eF : 0.f;
+      // without ALiBi (and with scale > 0) the maximum is taken on the raw
+      // scores and the scale folds into the exponent's FFMA
+      const bool direct = a.alibi == nullptr && c > 0.f;
+      const float cc = direct ? c : 1.f;
+      bool ok = true;
+      float m_run = -INFINITY, l_run = 0.f;
+      const int n = T.count();
+      for (int cix = 0; ok && cix < n; ++cix) {
+        const int j = T.jlo + cix;
+        ok = __all_sync(0xffffffffu, wait_or_abort(&bars[C::B_SF + qi], sm_s & 1, abort_flag));
+        if (!ok) break;
+        ++sm_s;
+        tc_fence_after();
+        uint32_t v[2][32];
+        tmem_ld32(s_col, v[0]);
+        tmem_ld32(s_col + 32, v[1]);
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&bars[C::B_SE + qi]);      // S_i may be overwritten now
+        const int key0 = j * kBN;
+        const bool full = key0 + kBN - 1 <= T.pos0 &&
+                          (a.window <= 0 || key0 >= T.last - a.window + 1);
+        const int nlo = full ? 0 : (row_ok ? lo_row - key0 : kBN);
+        const int nhi = full ? kBN - 1 : (row_ok ? pos - key0 : -1);
+        const float b0 = slope * static_cast<float>(key0 - pos);
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+          if (!direct) {
+#pragma unroll
+            for (int x = 0; x < 32; ++x)
+              v[h2][x] = __float_as_uint(fmaf(__uint_as_float(v[h2][x]), c,
+                                              fmaf(slope, static_cast<float>(32 * h2 + x), b0)));
+          }
+          if (!full) {
+#pragma unroll
+            for (int x = 0; x < 32; ++x)
+              if (32 * h2 + x < nlo || 32 * h2 + x > nhi) v[h2][x] = __float_as_uint(-INFINITY);
+          }
+#pragma unroll
+          for (int x2 = 0; x2 < 16; ++x2)
+            m4[x2 & 3] = fmax3(m4[x2 & 3], __uint_as_float(v[h2][2 * x2]),
+                               __uint_as_float(v[h2][2 * x2 + 1]));
+        }
+        float m_tile = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        if (direct) m_tile *= c;                 // scale > 0: the maximum commutes with it
+        const bool raise = (m_run == -INFINITY) ? (m_tile != -INFINITY)
+                                                : (m_tile > m_run + kRescaleGap);
+        const float m_new = raise ? m_tile : m_run;
+        const float alpha = (!raise || m_run == -INFINITY) ? 1.f : fast_exp2(m_run - m_new);
+        l_run *= alpha;
+        const float nmu = (m_new == -INFINITY) ? 0.f : -m_new;
+        // p = 2^(x - m_new) as 16-bit hi + lo pairs: for each 16 keys, 8
+        // columns of hi pairs then 8 of lo pairs
+        uint32_t pk[2][32];
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int h2 = 0; h2 < 2; ++h2) {
+#pragma unroll
+          for (int x2 = 0; x2 < 16; ++x2) {
+            const float p0 = fast_exp2(fmaf(__uint_as_float(v[h2][2 * x2]), cc, nmu));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(v[h2][2 * x2 + 1]), cc, nmu));
+            ls[x2 & 3] += p0 + p1;
+            const uint32_t hw = pack2<BF16>(p0, p1);
+            const int grp = x2 >> 3, w = x2 & 7;   // 16-key group within the half, pair
+            pk[h2][16 * grp + w] = hw;
+            pk[h2][16 * grp + 8 + w] =
+                pack2<BF16>(p0 - lo_half_to_float<BF16>(hw), p1 - lo_half_to_float<BF16>(hw >> 16));
+          }
+        }
+        l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        m_run = m_new;
+        if (cix > 0) {
+          // P_i and O_i are free once PV_i of the previous tile has completed
+          ok = __all_sync(0xffffffffu, wait_or_abort(&bars[C::B_PVD + qi], sm_p & 1, abort_flag));
+          if (!ok) break;
+          ++sm_p;
+          tc_fence_after();
+          if (__any_sync(0xffffffffu, raise && alpha != 1.f)) {
+#pragma unroll 1
+            for (int q2 = 0; q2 < D / 32; ++q2) {
+              uint32_t o[32];
+              tmem_ld32(o_col + 32 * q2, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tmem_st32(o_col + 32 * q2, o);
+            }
+          }
+        }
+        tmem_st32(p_col, pk[0]);
+        tmem_st32(p_col + 32, pk[1]);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars[C::B_PF + qi]);
+      }
+      // -------- epilogue: O_i row / l -> out
+      if (n > 0) {
+        const bool have = __all_sync(
+            0xffffffffu, ok && wait_or_abort(&bars[C::B_PVD + qi], sm_p & 1, abort_flag));
+        ++sm_p;
+        if (have) {
+          tc_fence_after();
+          const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+          const int64_t orow = (static_cast<int64_t>(U.cu0 + (NQ * U.pair + qi) * tq + row) *
+                                    a.num_q_heads + hq0 + g) * D;
+#pragma unroll 1
+          for (int q2 = 0; q2 < D / 32; ++q2) {
+            uint32_t o[32];
+            tmem_ld32(o_col + 32 * q2, o);
+            tmem_wait_ld();
+            if (!row_ok) continue;
+            if (a.out_dtype == 3) {
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow + 32 * q2);
+#pragma unroll
+              for (int e = 0; e < 8; ++e)
+                dst[e] = make_float4(__uint_as_float(o[4 * e]) * inv_l,
+                                     __uint_as_float(o[4 * e + 1]) * inv_l,
+                                     __uint_as_float(o[4 * e + 2]) * inv_l,
+                                     __uint_as_float(o[4 * e + 3]) * inv_l);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(a.out) + orow + 32 * q2);
+              const bool ob = (a.out_dtype == 1);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                uint32_t w[4];
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                  const float x0 = __uint_as_float(o[8 * e + 2 * x]) * inv_l;
+                  const float x1 = __uint_as_float(o[8 * e + 2 * x + 1]) * inv_l;
+                  w[x] = ob ? pack2<true>(x0, x1) : pack2<false>(x0, x1);
+                }
+                dst[e] = make_uint4(w[0], w[1], w[2], w[3]);
+              }
+            }
           }
         }
       }
     }
+    // ---- the V tiles every role counted for this unit
+
+    // ---- next unit: thread 0 takes it before the CTA-wide hand-over
+    if (threadIdx.x == 0) unit_slot[(k + 1) & 1] = atomicAdd(unit_counter, 1);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
   }
 
   // ---- teardown: every MMA and copy of this CTA has completed (or been
   // given a bounded chance to) before TMEM is released.
+  if (warp >= C::kMmaWarp0) {
+    tc_commit_warp(&bars[C::B_DR + (warp - C::kMmaWarp0)]);
+    (void)mbar_wait_bounded(&bars[C::B_DR + (warp - C::kMmaWarp0)], 0);
+  }
+  if ((warp == C::kKWarp || warp == C::kVWarp) && lane == 0 && *abort_flag) {
+    const bool is_v = warp == C::kVWarp;
+    const int nst = is_v ? C::kVSt : C::kKSt;
+    uint64_t* full = &bars[is_v ? C::B_VF : C::B_KF];
+    const uint32_t cnt = is_v ? vcnt : kcnt;
+    for (uint32_t s = 0; s < static_cast<uint32_t>(nst) && s < cnt; ++s)
+      (void)mbar_wait_bounded(&full[(cnt - 1 - s) % nst], ((cnt - 1 - s) / nst) & 1, 1u << 16);
+  }
   tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == C::kMmaWarp0) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
 }
 
-// Compact list of (request, query tile) items of the q_len >= 2 requests,
-// ordered by the number of key tiles each visits, most first (longest
-// processing time first: the heavy CTAs start in the first wave instead of
-// forming the grid's tail).  One CTA: a histogram of item weights in shared
-// memory, a descending exclusive scan over it, then each item takes a slot in
-// its weight's range (order within one weight is arbitrary; every item
-// writes its own output rows, so the result does not depend on it).
+// Compact list of (request, pair of query tiles) items of the q_len >= 2
+// requests, ordered by the number of key tiles the pair visits, most first
+// (longest processing time first: the heavy units are taken first instead of
+// forming the tail).  One CTA: a histogram of item weights in shared memory, a
+// descending exclusive scan over it, then each item takes a slot in its
+// weight's range (order within one weight is arbitrary; every item writes its
+// own output rows, so the result does not depend on it).  Also resets the
+// persistent kernel's unit counter.
 constexpr int kItemThreads = 1024;
 constexpr int kWeightBuckets = 4096;     // weights past the last bucket share it
 
 __device__ __forceinline__ int item_weight(const int32_t* cu, const int32_t* seqlens_k,
                                            int32_t max_context_len, int32_t window, int tq,
-                                           int r, int qt) {
+                                           int nq, int r, int pair) {
   const int q_len = cu[r + 1] - cu[r];
   const int kv_len = min(seqlens_k[r], max_context_len);
-  const int rows = min(tq, q_len - qt * tq);
-  const int pos0 = kv_len - q_len + qt * tq;
-  const int last = pos0 + rows - 1;
-  if (rows <= 0 || last < 0) return 0;
-  const int jlo = window > 0 ? max(0, pos0 - window + 1) / kBN : 0;
-  return min(last / kBN + 1 - jlo, kWeightBuckets - 1);
+  int w = 0;
+  for (int i = 0; i < nq; ++i) w += qtile(q_len, kv_len, tq, nq * pair + i, window).count();
+  return min(w, kWeightBuckets - 1);
 }
 
 __global__ void __launch_bounds__(kItemThreads)
 prefill_items_kernel(int32_t num_seqs, const int32_t* cu, const int32_t* seqlens_k,
-                     int32_t max_context_len, int32_t window, int tq, int2* items,
-                     int32_t* count, int32_t capacity) {
+                     int32_t max_context_len, int32_t window, int tq, int nq, int2* items,
+                     int32_t* count, int32_t capacity, int32_t* unit_counter) {
   __shared__ int s_hist[kWeightBuckets];
   __shared__ int s_part[kItemThreads];
   for (int i = threadIdx.x; i < kWeightBuckets; i += kItemThreads) s_hist[i] = 0;
   __syncthreads();
+  const int span = tq * nq;                // query positions per item
   // ---- histogram of item weights
   for (int r = threadIdx.x; r < num_seqs; r += kItemThreads) {
     const int ql = cu[r + 1] - cu[r];
     if (ql < 2) continue;
-    for (int qt = 0; qt < (ql + tq - 1) / tq; ++qt)
-      atomicAdd(&s_hist[item_weight(cu, seqlens_k, max_context_len, window, tq, r, qt)], 1);
+    for (int p = 0; p < (ql + span - 1) / span; ++p)
+      atomicAdd(&s_hist[item_weight(cu, seqlens_k, max_context_len, window, tq, nq, r, p)], 1);
   }
   __syncthreads();
   // ---- descending exclusive scan: bucket w starts after every heavier item.
-  // Thread t owns buckets kWeightBuckets-1-4t .. -3 (4 per thread, heaviest first).
   constexpr int kPer = kWeightBuckets / kItemThreads;
   int mine[kPer], sum = 0;
 #pragma unroll
@@ -550,38 +657,60 @@ prefill_items_kernel(int32_t num_seqs, const int32_t* cu, const int32_t* seqlens
   for (int r = threadIdx.x; r < num_seqs; r += kItemThreads) {
     const int ql = cu[r + 1] - cu[r];
     if (ql < 2) continue;
-    for (int qt = 0; qt < (ql + tq - 1) / tq; ++qt) {
-      const int slot =
-          atomicAdd(&s_hist[item_weight(cu, seqlens_k, max_context_len, window, tq, r, qt)], 1);
-      if (slot < capacity) items[slot] = make_int2(r, qt);
+    for (int p = 0; p < (ql + span - 1) / span; ++p) {
+      const int slot = atomicAdd(
+          &s_hist[item_weight(cu, seqlens_k, max_context_len, window, tq, nq, r, p)], 1);
+      if (slot < capacity) items[slot] = make_int2(r, p);
     }
   }
-  if (threadIdx.x == 0) *count = min(total, capacity);
+  if (threadIdx.x == 0) {
+    *count = min(total, capacity);
+    *unit_counter = 0;
+  }
 }
 
-template <bool BF16, int G>
+int g_num_sms[64];
+
+int num_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (g_num_sms[dev] <= 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    g_num_sms[dev] = n;
+  }
+  return g_num_sms[dev];
+}
+
+int ilog2(int x) {
+  int l = 0;
+  while ((1 << l) < x) ++l;
+  return l;
+}
+
+template <bool BF16, int D>
 cudaError_t launch_prefill_typed(const AttnArgs& a, const CUtensorMap& k, const CUtensorMap& v,
-                                 const CUtensorMap& q, int capacity, cudaStream_t s) {
-  auto kern = paged_prefill_kernel<BF16, G>;
-  const int64_t grid = static_cast<int64_t>(capacity) * a.num_kv_heads;
-  if (grid == 0) return cudaSuccess;
-  // the shared-memory limit is a per-device setting of the function: set it
-  // for the current device on every launch (a host-side call)
-  cudaError_t e =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+                                 const CUtensorMap& q, int capacity, int32_t* unit_counter,
+                                 cudaStream_t s) {
+  using C = Cfg<D>;
+  auto kern = paged_prefill_kernel<BF16, D>;
+  const int64_t units = static_cast<int64_t>(capacity) * a.num_kv_heads;
+  if (units == 0) return cudaSuccess;
+  cudaError_t e = ensure_smem_attribute(reinterpret_cast<const void*>(kern), C::kSmem);
   if (e != cudaSuccess) return e;
-  kern<<<static_cast<unsigned>(grid), kPfThreads, kSmemBytes, s>>>(a, k, v, q);
+  const int grid = static_cast<int>(units < num_sms() ? units : num_sms());
+  kern<<<grid, C::kThreads, C::kSmem, s>>>(a, k, v, q, ilog2(a.group), unit_counter);
   return cudaGetLastError();
 }
 
 template <bool BF16>
-cudaError_t launch_prefill_g(const AttnArgs& a, const CUtensorMap& k, const CUtensorMap& v,
-                             const CUtensorMap& q, int capacity, cudaStream_t s) {
-  switch (a.group) {
-    case 1: return launch_prefill_typed<BF16, 1>(a, k, v, q, capacity, s);
-    case 2: return launch_prefill_typed<BF16, 2>(a, k, v, q, capacity, s);
-    case 4: return launch_prefill_typed<BF16, 4>(a, k, v, q, capacity, s);
-    case 8: return launch_prefill_typed<BF16, 8>(a, k, v, q, capacity, s);
+cudaError_t launch_prefill_d(const AttnArgs& a, const CUtensorMap& k, const CUtensorMap& v,
+                             const CUtensorMap& q, int capacity, int32_t* ctr, cudaStream_t s) {
+  switch (a.head_dim) {
+    case 64: return launch_prefill_typed<BF16, 64>(a, k, v, q, capacity, ctr, s);
+    case 128: return launch_prefill_typed<BF16, 128>(a, k, v, q, capacity, ctr, s);
+    case 256: return launch_prefill_typed<BF16, 256>(a, k, v, q, capacity, ctr, s);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -589,29 +718,34 @@ cudaError_t launch_prefill_g(const AttnArgs& a, const CUtensorMap& k, const CUte
 }  // namespace
 
 bool prefill_supported(int q_dtype, int kv_dtype, int32_t head_dim, int32_t group) {
-  if (head_dim != 128) return false;
+  if (head_dim != 64 && head_dim != 128 && head_dim != 256) return false;
   if (!(kv_dtype == 0 || kv_dtype == 1) || q_dtype != kv_dtype) return false;
-  return group == 1 || group == 2 || group == 4 || group == 8;
+  return group >= 1 && group <= 128 && (group & (group - 1)) == 0;
 }
 
 int prefill_query_tile(int32_t group) { return 128 / group; }
 
+int prefill_tiles_per_item(int32_t head_dim) { return head_dim == 256 ? 1 : 2; }
+
 int32_t prefill_item_capacity(int32_t num_seqs, int32_t total_q) {
-  // sum_r ceil(q_len_r / tq) over requests with q_len_r >= 2, tq >= 16
-  return total_q / 16 + (num_seqs < total_q / 2 ? num_seqs : total_q / 2) + 1;
+  // every item holds at least one query row of a request with q_len >= 2
+  (void)num_seqs;
+  return total_q;
 }
 
 cudaError_t launch_paged_prefill(const AttnArgs& a, const CUtensorMap& kmap,
                                  const CUtensorMap& vmap, const CUtensorMap& qmap,
-                                 int32_t capacity, cudaStream_t stream) {
+                                 int32_t capacity, int32_t* unit_counter, cudaStream_t stream) {
   const int tq = 128 / a.group;
+  const int nq = prefill_tiles_per_item(a.head_dim);
   prefill_items_kernel<<<1, kItemThreads, 0, stream>>>(
-      a.num_seqs, a.cu_seqlens_q, a.seqlens_k, a.max_context_len, a.window, tq,
-      const_cast<int2*>(a.pf_items), const_cast<int32_t*>(a.pf_count), capacity);
+      a.num_seqs, a.cu_seqlens_q, a.seqlens_k, a.max_context_len, a.window, tq, nq,
+      const_cast<int2*>(a.pf_items), const_cast<int32_t*>(a.pf_count), capacity, unit_counter);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return a.kv_dtype == 1 ? launch_prefill_g<true>(a, kmap, vmap, qmap, capacity, stream)
-                         : launch_prefill_g<false>(a, kmap, vmap, qmap, capacity, stream);
+  return a.kv_dtype == 1 ? launch_prefill_d<true>(a, kmap, vmap, qmap, capacity, unit_counter, stream)
+                         : launch_prefill_d<false>(a, kmap, vmap, qmap, capacity, unit_counter,
+                                                   stream);
 }
 
 }  // namespace pa

@@ -69,6 +69,8 @@ def load_library(path: str = LIB_PATH):
     lib.pa_decode.restype = E
     lib.pa_varlen_workspace_size.argtypes = [i32, i32, i32, i32, i32]
     lib.pa_varlen_workspace_size.restype = sz
+    lib.pa_varlen_workspace_size_ex.argtypes = [i32, i32, i32, i32, i32, i32, i32, E, E]
+    lib.pa_varlen_workspace_size_ex.restype = sz
     lib.pa_varlen.argtypes = [P, E, P, E, i32, i32, i32, P, P, i32, i32, P, P, D, P, i32, F, P,
                               sz, P]
     lib.pa_varlen.restype = E
@@ -85,6 +87,8 @@ def load_library(path: str = LIB_PATH):
     lib.pa_copy_blocks.restype = E
     lib.pa_swap_blocks.argtypes = [P, P, P, P, D, i64, i64, P, i64, P]
     lib.pa_swap_blocks.restype = E
+    lib.pa_selftest_wait_timeout.argtypes = [P]
+    lib.pa_selftest_wait_timeout.restype = E
     lib.pa_hbm_read_probe.argtypes = [P, i64, P, P]
     lib.pa_hbm_read_probe.restype = E
     if path == LIB_PATH:
@@ -206,6 +210,16 @@ def pa_varlen_workspace_size(num_seqs: int, total_q: int, num_q_heads: int, head
                                                        max_context_len))
 
 
+def pa_varlen_workspace_size_ex(num_seqs: int, total_q: int, num_q_heads: int,
+                                num_kv_heads: int, head_dim: int, max_q_len: int,
+                                max_context_len: int, q_dtype: int, kv_dtype: int) -> int:
+    """Workspace for exactly these sizes and dtype codes (PA_F16 / PA_BF16 /
+    PA_FP8_E4M3): split-K partials only for the rows the decode kernel runs."""
+    return int(load_library().pa_varlen_workspace_size_ex(
+        num_seqs, total_q, num_q_heads, num_kv_heads, head_dim, max_q_len, max_context_len,
+        q_dtype, kv_dtype))
+
+
 def _workspace(nbytes: int, device, workspace: Optional[torch.Tensor]):
     if nbytes == 0:
         return workspace, 0 if workspace is None else workspace.numel()
@@ -271,7 +285,11 @@ def pa_varlen(out: torch.Tensor, q: torch.Tensor, cu_seqlens_q: torch.Tensor,
     total_q, hq, d = q.shape
     S = seqlens_k.shape[0]
     lib = load_library()
-    need = lib.pa_varlen_workspace_size(S, total_q, hq, d, max_context_len)
+    need = lib.pa_varlen_workspace_size_ex(S, total_q, hq, k_cache.shape[1], d, int(max_q_len),
+                                           max_context_len, dtype_code(q.dtype),
+                                           dtype_code(k_cache.dtype))
+    if out.data_ptr() % 16:
+        need = lib.pa_varlen_workspace_size(S, total_q, hq, d, max_context_len)
     workspace, wbytes = _workspace(need, q.device, workspace)
     desc = cache_desc(k_cache, k_scale, v_scale)
     args = (_ptr(out), dtype_code(out.dtype), _ptr(q), dtype_code(q.dtype), total_q, S, hq,
@@ -295,6 +313,12 @@ def pa_hbm_read_probe(buf: torch.Tensor, sink: torch.Tensor, stream=None) -> Non
     st = load_library().pa_hbm_read_probe(_ptr(buf), buf.numel() * buf.element_size(),
                                           _ptr(sink), _stream(stream))
     _check(st, "pa_hbm_read_probe")
+
+
+def pa_selftest_wait_timeout(stream=None) -> None:
+    """Enqueue the library's bounded-wait self-test: the next pa_device_error
+    returns PA_ERR_TIMEOUT (6)."""
+    _check(load_library().pa_selftest_wait_timeout(_stream(stream)), "pa_selftest_wait_timeout")
 
 
 def pa_device_error(stream=None) -> int:

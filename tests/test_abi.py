@@ -42,6 +42,26 @@ def test_status_strings(lib):
     assert pa.pa_status_string(99) == "PA_ERR_UNKNOWN"
 
 
+def test_varlen_workspace_ex_sizes_partials_for_the_rows_that_use_them(lib):
+    """With the chunk path (16-bit KV, head_dim 128, power-of-two group) only
+    the q_len-1 requests take split-K partials, one row each: the exact-type
+    size equals the worst-case size recomputed with num_seqs rows.  An E4M3
+    pool sends every row to the decode kernel, so the sizes agree."""
+    S, T, H, D, L = 204, 2248, 32, 128, 4097
+    worst = pa.pa_varlen_workspace_size(S, T, H, D, L)
+    chunk = pa.pa_varlen_workspace_size_ex(S, T, H, 8, D, 512, L, pa.PA_BF16, pa.PA_BF16)
+    fp8 = pa.pa_varlen_workspace_size_ex(S, T, H, 8, D, 512, L, pa.PA_BF16, pa.PA_FP8_E4M3)
+    decode_only = pa.pa_varlen_workspace_size_ex(S, T, H, 8, D, 1, L, pa.PA_BF16, pa.PA_BF16)
+    assert fp8 == worst == decode_only
+    assert chunk < 40e6 < worst
+    # partials of 204 rows x 32 heads x 9 parts (512 tokens) for m, l and o
+    al = lambda x: -(-x // 256) * 256  # noqa: E731
+    n = S * H * 9
+    head = 2 * al(4 * T) + al(8 * T) + 256
+    assert chunk == head + 2 * al(4 * n) + al(4 * n * D)
+    assert pa.pa_varlen_workspace_size_ex(S, T, H, 3, D, 512, L, pa.PA_BF16, pa.PA_BF16) == 0
+
+
 def test_decode_workspace_size_closed_form(lib):
     # one partition (no split) needs no workspace
     assert pa.pa_decode_workspace_size(64, 40, 128, 512, 512) == 0
@@ -86,8 +106,8 @@ def test_host_validation_rejects_before_any_launch(lib):
     # q heads not a multiple of kv heads
     assert lib.pa_decode(fake, 0, fake, 0, 4, 3, fake, fake, ctypes.byref(desc), fake, 8, fake,
                          100, 0.125, 0, None, 0, None) == 1
-    # group of 16 heads is not built
-    assert lib.pa_decode(fake, 0, fake, 0, 4, 32, fake, fake, ctypes.byref(desc), fake, 8, fake,
+    # a group of more than 128 query heads per KV head is not built
+    assert lib.pa_decode(fake, 0, fake, 0, 4, 512, fake, fake, ctypes.byref(desc), fake, 8, fake,
                          100, 0.125, 0, None, 0, None) == 2
     # q dtype differs from a 16-bit pool
     assert lib.pa_decode(fake, 0, fake, 1, 4, 2, fake, fake, ctypes.byref(desc), fake, 8, fake,

@@ -104,8 +104,9 @@ def test_decode_block_sizes(oracle, bs, hq, hkv, D):
 
 
 @pytest.mark.parametrize("bs", [8, 32])
-def test_decode_fp8_block_sizes(oracle, bs):
-    W = wl.build_workload("bs8", 510 + bs, np.ones(4, np.int64), [5, 40, 700, 1111], 8, 2, 128,
+@pytest.mark.parametrize("D", [64, 128])
+def test_decode_fp8_block_sizes(oracle, bs, D):
+    W = wl.build_workload("bs8", 510 + bs + D, np.ones(4, np.int64), [5, 40, 700, 1111], 8, 2, D,
                           kv_dtype=wl.FP8_E4M3, block_size=bs)
     _run_small(oracle, W, F32)
 
@@ -119,7 +120,7 @@ def test_varlen_block_sizes(oracle, bs):
         _run_small(oracle, W, F32)
 
 
-@pytest.mark.parametrize("D", [128, 256])
+@pytest.mark.parametrize("D", [64, 128, 256])
 @pytest.mark.parametrize("q_dtype", [wl.BF16, wl.F16])
 def test_decode_fp8_pool(oracle, D, q_dtype):
     W = wl.build_workload("fp8", 300 + D, np.ones(6, np.int64), [1, 17, 100, 513, 1024, 2000], 8,
@@ -128,7 +129,7 @@ def test_decode_fp8_pool(oracle, D, q_dtype):
         _run_small(oracle, W, out_dtype)
 
 
-@pytest.mark.parametrize("D", [128, 256])
+@pytest.mark.parametrize("D", [64, 128, 256])
 @pytest.mark.parametrize("q_dtype", [wl.BF16, wl.F16])
 def test_decode_fp8_query_dynamic_range(oracle, D, q_dtype):
     """E4M3 pool: the query enters QK^T as E4M3 hi + lo parts of q * 2^e, one
@@ -346,6 +347,46 @@ def test_out_of_range_slot_is_skipped_and_reported():
     bad = torch.tensor([W.num_blocks * 16 + 3], dtype=torch.int64, device="cuda")
     pa.pa_reshape_and_cache(d.new_k, d.new_v, bad, d.k_cache, d.v_cache)
     assert pa.pa_device_error() == 4
+
+
+def test_row_longer_than_max_context_len_is_cut_and_reported(oracle):
+    """A context_lens / seqlens_k entry above the promised max_context_len is
+    cut to max_context_len keys and reported as PA_ERR_OUT_OF_RANGE."""
+    W = wl.build_workload("cut", 12, np.ones(3, np.int64), [100, 300, 150], 4, 2, 64)
+    d = DeviceStep(W, out_dtype=F32)
+    d.fill_cache()
+    d.write_new()
+    torch.cuda.synchronize()
+    kc, vc = oracle_pools(oracle, W)
+    cut = 200
+    pa.pa_decode(d.out, d.q, d.k_cache, d.v_cache, d.block_tables, d.seqlens_k, cut, W.scale,
+                 partition_size=64, workspace=None)
+    assert pa.pa_device_error() == 4
+    want = oracle.paged_attention(W.q, W.q_dtype, W.cu_seqlens_q,
+                                  np.minimum(W.seqlens_k, cut).astype(np.int32), kc, vc,
+                                  W.kv_dtype, W.block_tables, W.scale)
+    assert_close(d.out_f64(), want, W, F32, "cut decode")
+    # the packed step: a request with q_len 2 and one with q_len 1, both too long
+    V = wl.build_workload("cutv", 13, [2, 1], [180, 300], 8, 2, 128)
+    e = DeviceStep(V, out_dtype=F32)
+    e.fill_cache()
+    e.write_new()
+    torch.cuda.synchronize()
+    kc, vc = oracle_pools(oracle, V)
+    pa.pa_varlen(e.out, e.q, e.cu, e.seqlens_k, V.max_q_len, 160, e.k_cache, e.v_cache,
+                 e.block_tables, V.scale)
+    assert pa.pa_device_error() == 4
+    assert torch.isfinite(e.out).all()
+
+
+def test_a_wait_that_runs_out_is_reported_and_the_context_survives(oracle):
+    """The bounded-wait path: a kernel whose wait can never complete gives up
+    after its limit, records PA_ERR_TIMEOUT and returns; the error word reads
+    back once, and the next attention call on the same context is correct."""
+    pa.pa_selftest_wait_timeout()
+    assert pa.pa_device_error() == 6
+    assert pa.pa_device_error() == 0
+    _run_small(oracle, wl.config(1), F32)
 
 
 def test_workspace_too_small_is_rejected():

@@ -1,10 +1,11 @@
-"""A NumPy model of the chunk kernel's arithmetic (CPU only): 128-key tiles,
-a running maximum raised only when a tile exceeds it by 2^8, P = 2^(x - m)
+"""A NumPy model of the chunk kernel's arithmetic (CPU only): 64-key tiles
+(as the kernel runs them; 128 too), a running maximum raised only when a tile exceeds it by 2^8, P = 2^(x - m)
 entering PV as a bf16 hi + lo pair, fp32 sums.  It pins the precision claim
 behind the hi + lo split against the exact fp64 result: with the pair the error is
 far inside the 2e-3 bound; with P as one bf16 value a row with a few large
 values leaves it."""
 import numpy as np
+import pytest
 
 from paged_kv_cache_lens_b200 import workloads as wl
 
@@ -51,19 +52,22 @@ def _bf16_normal(rng, shape, sigma=1.0):
     return _bf16((rng.standard_normal(shape) * sigma).astype(np.float32))
 
 
-def test_hi_lo_split_stays_far_inside_the_bound():
+@pytest.mark.parametrize("tile", [64, 128])
+def test_hi_lo_split_stays_far_inside_the_bound(tile):
     rng = np.random.default_rng(11)
     D = 128
     scale = D ** -0.5
     worst = 0.0
-    for L in (1, 2, 3, 17, 128, 129, 700, 2000):
+    for L in (1, 2, 3, 17, 64, 65, 128, 129, 700, 2000):
         K, V = _bf16_normal(rng, (L, D)), _bf16_normal(rng, (L, D))
         q = _bf16_normal(rng, D)
-        worst = max(worst, np.abs(model_row(q, K, V, scale) - exact_row(q, K, V, scale)).max())
+        err = np.abs(model_row(q, K, V, scale, tile=tile) - exact_row(q, K, V, scale)).max()
+        worst = max(worst, err)
     assert worst < 2e-5
 
 
-def test_lazy_rescale_handles_a_late_large_maximum():
+@pytest.mark.parametrize("tile", [64, 128])
+def test_lazy_rescale_handles_a_late_large_maximum(tile):
     """A key in the last tile scores far above every earlier one: the running
     maximum must be raised and O and l rescaled, not overflow."""
     rng = np.random.default_rng(12)
@@ -71,7 +75,7 @@ def test_lazy_rescale_handles_a_late_large_maximum():
     K, V = _bf16_normal(rng, (L, D)), _bf16_normal(rng, (L, D))
     q = _bf16_normal(rng, D)
     K[590] = _bf16(q * 8)                                       # score ~ 8 |q|^2 / sqrt(D)
-    got = model_row(q, K, V, D ** -0.5)
+    got = model_row(q, K, V, D ** -0.5, tile=tile)
     assert np.isfinite(got).all()
     assert np.abs(got - exact_row(q, K, V, D ** -0.5)).max() < 2e-5
 

@@ -137,3 +137,4 @@ def test_bf16_decode_is_upper_half_of_binary32(oracle):
             assert v == want
     assert oracle.bf16_to_double(0x3F80) == 1.0
     assert oracle.bf16_to_double(0x4049) == 3.140625
+

@@ -80,6 +80,25 @@ def test_static_scratch_matches_pa_decode_on_two_calls(lib):
         torch.testing.assert_close(out, ref, rtol=0, atol=2e-3)
 
 
+def test_static_scratch_call_takes_no_device_memory(lib):
+    """After the first call (which loads the library's device code, array
+    included), a call leaves the device's free memory exactly as it found it:
+    it allocates nothing."""
+    torch.cuda.set_device(0)
+    W, kc, vc, q, bt, sk = _setup(74, 32, 256)
+    out = torch.empty((W.num_seqs, W.num_q_heads, W.head_dim), dtype=torch.float32,
+                      device="cuda")
+    assert _call_static(lib, out, q, kc, vc, bt, sk, W, 256) == 0
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        assert _call_static(lib, out, q, kc, vc, bt, sk, W, 256) == 0
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+    assert pa.pa_device_error() == 0
+
+
 def test_static_scratch_rejects_sizes_beyond_its_capacity(lib):
     torch.cuda.set_device(0)
     W, kc, vc, q, bt, sk = _setup(73, 4, 128)
