@@ -256,11 +256,15 @@ TD_NAMES = {wl.F16: "float16", wl.BF16: "bfloat16", wl.F32: "float32"}
 
 def chunk_path(W) -> bool:
     """Whether pa_varlen sends this step's q_len >= 2 requests to the
-    tensor-core chunk kernel (the library's rule: 16-bit KV and q of one type,
-    head_dim 128, GQA group 1, 2, 4 or 8)."""
+    tensor-core chunk kernel (the library's rule: a power-of-two GQA group up
+    to 128; a 16-bit pool with q of its type at head_dim 64, 128 or 256, or an
+    E4M3 pool at head_dim 128)."""
     g = W.num_q_heads // W.num_kv_heads
-    return (not W.decode and W.max_q_len >= 2 and W.kv_dtype in (wl.F16, wl.BF16)
-            and W.q_dtype == W.kv_dtype and W.head_dim == 128 and g in (1, 2, 4, 8))
+    if W.decode or W.max_q_len < 2 or g < 1 or g > 128 or (g & (g - 1)):
+        return False
+    if W.kv_dtype == wl.FP8_E4M3:
+        return W.head_dim == 128
+    return W.q_dtype == W.kv_dtype and W.head_dim in (64, 128, 256)
 
 
 class DeviceWorkload:

@@ -41,13 +41,12 @@ namespace {
 
 constexpr int kBN = 64;                  // keys per tile
 constexpr int kTblMax = 2048;            // block-table entries cached in shared memory
-constexpr uint32_t kWaitLimit = 1u << 15;      // hinted waits of up to 50 us each: ~1.6 s
-constexpr uint32_t kWaitHintNs = 50000;
+constexpr uint32_t kWaitLimit = 1u << 21;
 constexpr float kRescaleGap = 8.f;       // raise the running max when exceeded by 2^8
 constexpr float kLog2eF = 1.4426950408889634f;
 constexpr uint32_t kTmemCols = 512;
 
-template <int D>
+template <int D, bool FP8 = false>
 struct Cfg {
   static constexpr int NQ = (D == 256) ? 1 : 2;            // query tiles per unit
   static constexpr int kCB = D / 64;                       // 128-byte column blocks
@@ -55,8 +54,12 @@ struct Cfg {
   static constexpr int kQBytes = kCB * kQCB;
   static constexpr int kKVCB = kBN * 128;                  // bytes of a K/V tile column block
   static constexpr int kKVBytes = kCB * kKVCB;
-  static constexpr int kKSt = (D == 256) ? 2 : 4;
-  static constexpr int kVSt = (D == 256) ? 2 : 4;
+  static constexpr int kKSt = (D == 256) ? 2 : (FP8 ? 3 : 4);
+  static constexpr int kVSt = (D == 256) ? 2 : (FP8 ? 3 : 4);
+  // E4M3 pools: tiles land in a byte staging ring and are widened to f16
+  // into the operand rings by their producer
+  static constexpr int kSt8 = FP8 ? 2 : 0;
+  static constexpr int kStage8Bytes = kBN * D;             // one E4M3 tile (128-byte rows)
   static constexpr int kSoftmaxWarps = 4 * NQ;
   static constexpr int kKWarp = kSoftmaxWarps;             // K producer
   static constexpr int kVWarp = kSoftmaxWarps + 1;         // V producer
@@ -65,14 +68,18 @@ struct Cfg {
   static constexpr int kQOff = 0;
   static constexpr int kKOff = NQ * kQBytes;
   static constexpr int kVOff = kKOff + kKSt * kKVBytes;
-  static constexpr int kTblOff = kVOff + kVSt * kKVBytes;
+  static constexpr int kK8Off = kVOff + kVSt * kKVBytes;
+  static constexpr int kV8Off = kK8Off + kSt8 * kStage8Bytes;
+  static constexpr int kTblOff = kV8Off + kSt8 * kStage8Bytes;
   static constexpr int kBarOff = kTblOff + kTblMax * 4;
   // barriers: Q full [NQ] | K full, empty [kKSt] | V full, empty [kVSt] |
-  //           S full, S free, P full, PV done [NQ] | drain [NQ] | V fixed
+  //           S full, S free, P full, PV done [NQ] | drain [NQ] | V fixed |
+  //           Q ready [NQ] | K, V staging full [kSt8] (E4M3 pools)
   static constexpr int B_Q = 0, B_KF = NQ, B_KE = B_KF + kKSt, B_VF = B_KE + kKSt,
                        B_VE = B_VF + kVSt, B_SF = B_VE + kVSt, B_SE = B_SF + NQ,
                        B_PF = B_SE + NQ, B_PVD = B_PF + NQ, B_DR = B_PVD + NQ,
-                       B_VX = B_DR + NQ, kBars = B_VX + 1;
+                       B_VX = B_DR + NQ, B_QR = B_VX + 1, B_K8 = B_QR + NQ,
+                       B_V8 = B_K8 + kSt8, kBars = B_V8 + kSt8;
   static constexpr int kMiscOff = kBarOff + kBars * 8;     // tmem base, abort, unit slots
   // + alignment slack; at least 116 KiB so that two CTAs never share an SM
   // (each allocates all 512 TMEM columns)
@@ -87,8 +94,8 @@ struct Cfg {
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity,
                                               volatile int* abort_flag) {
   for (uint32_t i = 0; i < kWaitLimit; ++i) {
-    if (mbar_try_wait_hint(bar, parity, kWaitHintNs)) return true;
-    if (*abort_flag) return false;
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 1023) == 1023 && *abort_flag) return false;
   }
   *abort_flag = 1;
   report_error(kErrTimeout);
@@ -162,12 +169,76 @@ __device__ __forceinline__ Unit<NQ> make_unit(const AttnArgs& a, int idx, int tq
   return u;
 }
 
-template <bool BF16, int D>
-__global__ void __launch_bounds__(Cfg<D>::kThreads, 1)
+// E4M3 pool tile staging -> f16 operand tile: 16 bytes (16 dims) of row r at
+// 128-byte-swizzled chunk c become 32 bytes (two 8-dim chunks) of the f16
+// tile's column block c / 4, also 128-byte swizzled.
+template <int D>
+__device__ __forceinline__ void widen_e4m3_tile(const uint8_t* src, uint8_t* dst, int lane) {
+  constexpr int kChunks = D / 16;                  // 16-byte chunks per E4M3 row
+  for (int ix = lane; ix < kBN * kChunks; ix += 32) {
+    const int r = ix / kChunks, c = ix % kChunks;
+    const int sw = r & 7;
+    const uint4 w = *reinterpret_cast<const uint4*>(src + (c >> 3) * (kBN * 128) + r * 128 +
+                                                    (((c & 7) ^ sw) << 4));
+    const uint4 lo = make_uint4(e4m3x2_to_f16x2(w.x), e4m3x2_to_f16x2(w.x >> 16),
+                                e4m3x2_to_f16x2(w.y), e4m3x2_to_f16x2(w.y >> 16));
+    const uint4 hi = make_uint4(e4m3x2_to_f16x2(w.z), e4m3x2_to_f16x2(w.z >> 16),
+                                e4m3x2_to_f16x2(w.w), e4m3x2_to_f16x2(w.w >> 16));
+    uint8_t* row = dst + (c >> 2) * (kBN * 128) + r * 128;
+    *reinterpret_cast<uint4*>(row + (((2 * (c & 3)) ^ sw) << 4)) = lo;
+    *reinterpret_cast<uint4*>(row + (((2 * (c & 3) + 1) ^ sw) << 4)) = hi;
+  }
+}
+
+// bf16 query tile -> f16, in place (128-byte rows, the swizzle is a
+// permutation of whole 16-byte chunks within a row, so it is kept).
+template <int D>
+__device__ __forceinline__ void q_bf16_to_f16(uint8_t* q, int lane) {
+  for (int ix = lane; ix < 128 * D / 8; ix += 32) {
+    uint4* p = reinterpret_cast<uint4*>(q) + ix;
+    uint4 w = *p;
+    w.x = bf16x2_to_f16x2(w.x);
+    w.y = bf16x2_to_f16x2(w.y);
+    w.z = bf16x2_to_f16x2(w.z);
+    w.w = bf16x2_to_f16x2(w.w);
+    *p = w;
+  }
+}
+
+// P = 2^(x - m) for the PV product as two 16-bit values per key.
+//  bf16 pools: hi = p truncated to bf16 (the upper half of its fp32 bits),
+//    lo = (p - hi) truncated the same way: p - (hi + lo) < 2^-14 p, no
+//    conversion instruction (the exponentials already keep the conversion
+//    pipe busy);
+//  f16 pools: hi = f16(p), lo = f16(p - hi), nearest even;
+//  E4M3 pools (5e-2 tolerance): hi = f16(p) alone, lo unused.
+template <int KVT>
+__device__ __forceinline__ void pack_p(float p0, float p1, uint32_t& hi, uint32_t& lo) {
+  if constexpr (KVT == 1) {
+    const uint32_t b0 = __float_as_uint(p0), b1 = __float_as_uint(p1);
+    hi = __byte_perm(b0, b1, 0x7632);
+    const float r0 = p0 - __uint_as_float(b0 & 0xFFFF0000u);
+    const float r1 = p1 - __uint_as_float(b1 & 0xFFFF0000u);
+    lo = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
+  } else if constexpr (KVT == 0) {
+    hi = pack2<false>(p0, p1);
+    lo = pack2<false>(p0 - lo_half_to_float<false>(hi), p1 - lo_half_to_float<false>(hi >> 16));
+  } else {
+    hi = pack2<false>(p0, p1);
+    lo = 0;
+  }
+}
+
+// KVT: 0 f16 pool, 1 bf16 pool, 2 E4M3 pool (widened to f16; the query is
+// bf16 when Q_BF16, converted to f16 in shared memory).
+template <int KVT, bool Q_BF16, int D>
+__global__ void __launch_bounds__(Cfg<D, KVT == 2>::kThreads, 1)
 paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CUtensorMap kmap,
                      const __grid_constant__ CUtensorMap vmap,
                      const __grid_constant__ CUtensorMap qmap, int log2g, int32_t* unit_counter) {
-  using C = Cfg<D>;
+  constexpr bool FP8 = (KVT == 2);
+  constexpr bool BF16 = (KVT == 1);                // the MMA operand type
+  using C = Cfg<D, FP8>;
   constexpr int NQ = C::NQ;
   constexpr uint32_t kIdescS = idesc_f16(BF16, 128, kBN, false);
   constexpr uint32_t kIdescPV = idesc_f16(BF16, 128, D, true);
@@ -204,8 +275,15 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
       mbar_init(&bars[C::B_VF + s], 1);
       mbar_init(&bars[C::B_VE + s], NQ);
     }
-    for (int i = 0; i < NQ; ++i) mbar_init(&bars[C::B_DR + i], 1);
+    for (int i = 0; i < NQ; ++i) {
+      mbar_init(&bars[C::B_DR + i], 1);
+      mbar_init(&bars[C::B_QR + i], 1);
+    }
     mbar_init(&bars[C::B_VX], 1);
+    for (int s = 0; s < C::kSt8; ++s) {
+      mbar_init(&bars[C::B_K8 + s], 1);
+      mbar_init(&bars[C::B_V8 + s], 1);
+    }
     *abort_flag = 0;
     unit_slot[0] = atomicAdd(unit_counter, 1);
     fence_barrier_init();
@@ -222,6 +300,10 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
   // Running counts of every barrier's completed phases, kept across units by
   // the roles that wait on them (parity = count & 1).
   uint32_t kcnt = 0, vcnt = 0;             // K / V tiles loaded (producers) or passed (others)
+  uint32_t c8 = 0;                         // producers (E4M3): tiles staged
+  uint32_t qc8[NQ];                        // K producer (E4M3): loads of each query tile
+#pragma unroll
+  for (int i = 0; i < NQ; ++i) qc8[i] = 0;
   uint32_t mq = 0, ms = 0, mp = 0, mx = 0; // MMA warp: its Q loads, S tiles, PV batches, V fixes
   uint32_t sm_s = 0, sm_p = 0;             // softmax group: its tile's S tiles and PV batches
 
@@ -265,6 +347,88 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
       const CUtensorMap* map = is_v ? &vmap : &kmap;
       uint8_t* ring = smem + (is_v ? C::kVOff : C::kKOff);
       uint32_t& cnt = is_v ? vcnt : kcnt;
+      if constexpr (FP8) {
+        // ---- E4M3 pool: TMA into the byte staging ring, widen to f16 into
+        // the operand ring, then release the operand stage
+        uint64_t* sfull = &bars[is_v ? C::B_V8 : C::B_K8];
+        uint8_t* stage = smem + (is_v ? C::kV8Off : C::kK8Off);
+        auto stage_tile = [&](int u) {         // lane 0 arms, lanes 0-3 load
+          const uint32_t s8 = (c8 + u) % C::kSt8;
+          if (lane == 0) mbar_arrive_expect_tx(&sfull[s8], C::kStage8Bytes);
+          __syncwarp();
+          if (lane < kBN / 16) {
+            const int sti = (U.j0 + u) * (kBN / 16) + lane;
+            int y0 = oob_row, y1 = bs == 8 ? oob_row : -1;
+            if (sti * 16 <= last_all) {
+              const int32_t* src = (sti + 1) * 16 / bs + 1 < kTblMax ? tbl : bt;
+              int r0, r1;
+              if (tile_rows(src, sti, bs, nblk, a.num_blocks, a.num_kv_heads, U.h, oob_row, r0,
+                            r1)) {
+                y0 = r0;
+                y1 = r1;
+              } else {
+                report_error(kErrBlockRange);
+              }
+            }
+            uint8_t* box = stage + s8 * C::kStage8Bytes + lane * 2048;
+#pragma unroll
+            for (int cb = 0; cb < D / 128; ++cb) {
+              tma_load_2d(box + cb * (kBN * 128), map, cb * 128, y0, &sfull[s8], pol);
+              if (y1 >= 0)
+                tma_load_2d(box + cb * (kBN * 128) + 1024, map, cb * 128, y1, &sfull[s8], pol);
+            }
+          }
+        };
+        for (int u = 0; u < C::kSt8 && u < U.nu; ++u) stage_tile(u);
+        if (!is_v) {
+          // the query tiles: f16 in shared memory before the MMA warps read them
+#pragma unroll
+          for (int i = 0; i < NQ; ++i) {
+            if (U.qt[i].rows <= 0) continue;
+            if (__all_sync(0xffffffffu,
+                           wait_or_abort(&bars[C::B_Q + i], qc8[i] & 1, abort_flag))) {
+              if constexpr (Q_BF16) q_bf16_to_f16<D>(smem + C::kQOff + i * C::kQBytes, lane);
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&bars[C::B_QR + i]);
+            }
+            ++qc8[i];
+          }
+        }
+        for (int u = 0; u < U.nu; ++u) {
+          const uint32_t s8 = (c8 + u) % C::kSt8;
+          const uint32_t st = cnt % nst;
+          bool go = __all_sync(0xffffffffu, wait_or_abort(&sfull[s8], ((c8 + u) / C::kSt8) & 1,
+                                                            abort_flag));
+          if (go && cnt >= static_cast<uint32_t>(nst))
+            go = __all_sync(0xffffffffu,
+                            wait_or_abort(&empty[st], ((cnt / nst) - 1) & 1, abort_flag));
+          if (!go) break;
+          uint8_t* dst = ring + st * C::kKVBytes;
+          widen_e4m3_tile<D>(stage + s8 * C::kStage8Bytes, dst, lane);
+          if (is_v && U.stale && u == U.nu - 1) {
+            // rows of the context's last 16-key block past kv_len: zero
+            const int jl = U.j0 + U.nu - 1;
+            const int r0 = U.kv_len - jl * kBN;
+            const int r1 = ((U.kv_len + 15) & ~15) - jl * kBN;
+            for (int ix = lane; ix < (r1 - r0) * 8 * C::kCB; ix += 32) {
+              const int rr = r0 + ix / (8 * C::kCB);
+              const int rem = ix % (8 * C::kCB);
+              *reinterpret_cast<uint4*>(dst + (rem >> 3) * C::kKVCB + rr * 128 + (rem & 7) * 16) =
+                  make_uint4(0, 0, 0, 0);
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&full[st]);
+          ++cnt;
+          __syncwarp();
+          if (u + C::kSt8 < U.nu) stage_tile(u + C::kSt8);
+        }
+        c8 += U.nu;
+        if (is_v && U.stale && lane == 0) mbar_arrive(&bars[C::B_VX]);
+        __syncwarp();
+      } else
       for (int u = 0; u < U.nu; ++u) {
         const int j = U.j0 + u;
         const uint32_t st = cnt % nst;
@@ -302,7 +466,7 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
         }
         ++cnt;
       }
-      if (is_v && U.stale && !*abort_flag) {
+      if (!FP8 && is_v && U.stale && !*abort_flag) {
         // V rows of the context's last 16-key block past kv_len hold whatever
         // the slots held; P is 0 there but 0 * NaN is NaN: once the unit's
         // last V tile (which holds them) has landed, clear them, then let
@@ -343,7 +507,7 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
       const uint64_t qdesc =
           smem_desc_sw128(smem_u32(smem + C::kQOff + i * C::kQBytes), 16, 1024);
       if (T.rows > 0) {
-        ok = wait_all(&bars[C::B_Q + i], mq & 1);
+        ok = wait_all(&bars[FP8 ? C::B_QR + i : C::B_Q + i], mq & 1);
         ++mq;
       }
       const uint64_t kdesc0 = smem_desc_sw128(smem_u32(smem + C::kKOff), 16, 1024);
@@ -393,7 +557,7 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
               // keys 16kk .. 16kk+15: 8 columns of hi pairs, then 8 of lo pairs
               const uint64_t vk = vd + static_cast<uint64_t>((kk * 2048) >> 4);
               tc_mma_ts_warp(d_o, a_p + 16 * kk, vk, kIdescPV, (first_pv && kk == 0) ? 0u : 1u);
-              tc_mma_ts_warp(d_o, a_p + 16 * kk + 8, vk, kIdescPV, 1u);
+              if constexpr (!FP8) tc_mma_ts_warp(d_o, a_p + 16 * kk + 8, vk, kIdescPV, 1u);
             }
             first_pv = false;
             tc_commit_warp(&bars[C::B_PVD + i]);
@@ -417,7 +581,7 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
       const uint32_t s_col = lane_base + C::kSCol + 64 * qi;
       const uint32_t p_col = lane_base + C::kPCol + 64 * qi;
       const uint32_t o_col = lane_base + C::kOCol + D * qi;
-      const float c = a.scale * kLog2eF;
+      const float c = a.scale * kLog2eF * (FP8 ? a.k_scale[U.h] : 1.f);
       const int lo_row = a.window > 0 ? pos - a.window + 1 : 0;
       const float slope = a.alibi ? a.alibi[hq0 + g] * kLog2eF : 0.f;
       // without ALiBi (and with scale > 0) the maximum is taken on the raw
@@ -483,11 +647,8 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
             const float p0 = fast_exp2(fmaf(__uint_as_float(v[h2][2 * x2]), cc, nmu));
             const float p1 = fast_exp2(fmaf(__uint_as_float(v[h2][2 * x2 + 1]), cc, nmu));
             ls[x2 & 3] += p0 + p1;
-            const uint32_t hw = pack2<BF16>(p0, p1);
             const int grp = x2 >> 3, w = x2 & 7;   // 16-key group within the half, pair
-            pk[h2][16 * grp + w] = hw;
-            pk[h2][16 * grp + 8 + w] =
-                pack2<BF16>(p0 - lo_half_to_float<BF16>(hw), p1 - lo_half_to_float<BF16>(hw >> 16));
+            pack_p<KVT>(p0, p1, pk[h2][16 * grp + w], pk[h2][16 * grp + 8 + w]);
           }
         }
         l_run += (ls[0] + ls[1]) + (ls[2] + ls[3]);
@@ -523,7 +684,8 @@ paged_prefill_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__
         ++sm_p;
         if (have) {
           tc_fence_after();
-          const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+          const float inv_l =
+              l_run > 0.f ? (FP8 ? a.v_scale[U.h] : 1.f) / l_run : 0.f;
           const int64_t orow = (static_cast<int64_t>(U.cu0 + (NQ * U.pair + qi) * tq + row) *
                                     a.num_q_heads + hq0 + g) * D;
 #pragma unroll 1
@@ -689,12 +851,12 @@ int ilog2(int x) {
   return l;
 }
 
-template <bool BF16, int D>
+template <int KVT, bool Q_BF16, int D>
 cudaError_t launch_prefill_typed(const AttnArgs& a, const CUtensorMap& k, const CUtensorMap& v,
                                  const CUtensorMap& q, int capacity, int32_t* unit_counter,
                                  cudaStream_t s) {
-  using C = Cfg<D>;
-  auto kern = paged_prefill_kernel<BF16, D>;
+  using C = Cfg<D, KVT == 2>;
+  auto kern = paged_prefill_kernel<KVT, Q_BF16, D>;
   const int64_t units = static_cast<int64_t>(capacity) * a.num_kv_heads;
   if (units == 0) return cudaSuccess;
   cudaError_t e = ensure_smem_attribute(reinterpret_cast<const void*>(kern), C::kSmem);
@@ -704,23 +866,33 @@ cudaError_t launch_prefill_typed(const AttnArgs& a, const CUtensorMap& k, const 
   return cudaGetLastError();
 }
 
-template <bool BF16>
+template <int KVT>
 cudaError_t launch_prefill_d(const AttnArgs& a, const CUtensorMap& k, const CUtensorMap& v,
                              const CUtensorMap& q, int capacity, int32_t* ctr, cudaStream_t s) {
+  constexpr bool QB = (KVT == 1);
   switch (a.head_dim) {
-    case 64: return launch_prefill_typed<BF16, 64>(a, k, v, q, capacity, ctr, s);
-    case 128: return launch_prefill_typed<BF16, 128>(a, k, v, q, capacity, ctr, s);
-    case 256: return launch_prefill_typed<BF16, 256>(a, k, v, q, capacity, ctr, s);
+    case 64: return launch_prefill_typed<KVT, QB, 64>(a, k, v, q, capacity, ctr, s);
+    case 128: return launch_prefill_typed<KVT, QB, 128>(a, k, v, q, capacity, ctr, s);
+    case 256: return launch_prefill_typed<KVT, QB, 256>(a, k, v, q, capacity, ctr, s);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_prefill_fp8(const AttnArgs& a, const CUtensorMap& k, const CUtensorMap& v,
+                               const CUtensorMap& q, int capacity, int32_t* ctr, cudaStream_t s) {
+  if (a.head_dim != 128) return cudaErrorInvalidValue;
+  return a.q_dtype == 1 ? launch_prefill_typed<2, true, 128>(a, k, v, q, capacity, ctr, s)
+                        : launch_prefill_typed<2, false, 128>(a, k, v, q, capacity, ctr, s);
 }
 
 }  // namespace
 
 bool prefill_supported(int q_dtype, int kv_dtype, int32_t head_dim, int32_t group) {
+  if (group < 1 || group > 128 || (group & (group - 1)) != 0) return false;
+  if (kv_dtype == 2)   // E4M3 pool, widened to f16 in shared memory: head_dim 128
+    return head_dim == 128 && (q_dtype == 0 || q_dtype == 1);
   if (head_dim != 64 && head_dim != 128 && head_dim != 256) return false;
-  if (!(kv_dtype == 0 || kv_dtype == 1) || q_dtype != kv_dtype) return false;
-  return group >= 1 && group <= 128 && (group & (group - 1)) == 0;
+  return (kv_dtype == 0 || kv_dtype == 1) && q_dtype == kv_dtype;
 }
 
 int prefill_query_tile(int32_t group) { return 128 / group; }
@@ -743,9 +915,9 @@ cudaError_t launch_paged_prefill(const AttnArgs& a, const CUtensorMap& kmap,
       const_cast<int2*>(a.pf_items), const_cast<int32_t*>(a.pf_count), capacity, unit_counter);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return a.kv_dtype == 1 ? launch_prefill_d<true>(a, kmap, vmap, qmap, capacity, unit_counter, stream)
-                         : launch_prefill_d<false>(a, kmap, vmap, qmap, capacity, unit_counter,
-                                                   stream);
+  if (a.kv_dtype == 2) return launch_prefill_fp8(a, kmap, vmap, qmap, capacity, unit_counter, stream);
+  return a.kv_dtype == 1 ? launch_prefill_d<1>(a, kmap, vmap, qmap, capacity, unit_counter, stream)
+                         : launch_prefill_d<0>(a, kmap, vmap, qmap, capacity, unit_counter, stream);
 }
 
 }  // namespace pa

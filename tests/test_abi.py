@@ -43,16 +43,20 @@ def test_status_strings(lib):
 
 
 def test_varlen_workspace_ex_sizes_partials_for_the_rows_that_use_them(lib):
-    """With the chunk path (16-bit KV, head_dim 128, power-of-two group) only
-    the q_len-1 requests take split-K partials, one row each: the exact-type
-    size equals the worst-case size recomputed with num_seqs rows.  An E4M3
-    pool sends every row to the decode kernel, so the sizes agree."""
+    """With the chunk path (a power-of-two group; a 16-bit pool at head_dim
+    64/128/256 or an E4M3 pool at 128) only the q_len-1 requests take split-K
+    partials, one row each: the exact-type size is the worst-case size
+    recomputed with num_seqs rows.  A step of decode rows only, or a q dtype
+    other than the pool's 16-bit type, sends every row to the decode kernel:
+    then the sizes agree."""
     S, T, H, D, L = 204, 2248, 32, 128, 4097
     worst = pa.pa_varlen_workspace_size(S, T, H, D, L)
     chunk = pa.pa_varlen_workspace_size_ex(S, T, H, 8, D, 512, L, pa.PA_BF16, pa.PA_BF16)
     fp8 = pa.pa_varlen_workspace_size_ex(S, T, H, 8, D, 512, L, pa.PA_BF16, pa.PA_FP8_E4M3)
+    mixed_types = pa.pa_varlen_workspace_size_ex(S, T, H, 8, D, 512, L, pa.PA_F16, pa.PA_BF16)
     decode_only = pa.pa_varlen_workspace_size_ex(S, T, H, 8, D, 1, L, pa.PA_BF16, pa.PA_BF16)
-    assert fp8 == worst == decode_only
+    assert mixed_types == worst == decode_only
+    assert fp8 == chunk
     assert chunk < 40e6 < worst
     # partials of 204 rows x 32 heads x 9 parts (512 tokens) for m, l and o
     al = lambda x: -(-x // 256) * 256  # noqa: E731

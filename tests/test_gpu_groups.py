@@ -4,7 +4,8 @@ paged kernels cover MHA, MQA and GQA): groups of more than 8 query heads per
 KV head (MQA 16/1, 32/1, 128/1; GQA 64/4 and a non-power-of-two 24/2) in
 decode and in the packed varlen step, the tensor-core chunk path at head_dim
 64 and 256, and a step with more chunk work units than the GPU has SMs (each
-persistent chunk CTA then runs several units).
+persistent chunk CTA then runs several units), and E4M3 pools on the chunk
+path (K and V widened to f16 in shared memory).
 """
 import math
 
@@ -115,3 +116,25 @@ def test_full_size_mqa_decode_sampled(oracle):
     ph = np.tile(np.arange(W.num_q_heads), len(rows))
     want = oracle_attention(oracle, W, kc, vc, pairs=(pr, ph), num_threads=8)
     assert_close(got[pr, ph], want, W, W.out_dtype, W.name)
+
+
+@pytest.mark.parametrize("hq,hkv", [(8, 2), (4, 4), (32, 8)])
+@pytest.mark.parametrize("q_dtype", [wl.BF16, wl.F16])
+def test_varlen_fp8_pool_on_the_chunk_path(oracle, hq, hkv, q_dtype):
+    """E4M3 pools at head_dim 128 run their chunks on the tensor-core kernel
+    (K and V widened to f16 in shared memory): chunks of several query tiles
+    over cached context off the block and key-tile grid, decode rows beside."""
+    q_lens = [300, 1, 130, 257, 2]
+    kv_lens = [300 + 77, 1000, 130 + 400, 257 + 129, 2 + 61]
+    W = wl.build_workload("v8c", 700 + hq + q_dtype, q_lens, kv_lens, hq, hkv, 128, dtype=q_dtype,
+                          kv_dtype=wl.FP8_E4M3, out_dtype=wl.BF16)
+    _run(oracle, W, F32)
+    _run(oracle, W, wl.BF16)
+
+
+def test_varlen_fp8_pool_chunks_window_alibi_and_block_sizes(oracle):
+    for bs in (8, 16, 32):
+        W = wl.build_workload("v8w", 720 + bs, [200, 1, 90], [200 + 300, 500, 90], 8, 2, 128,
+                              kv_dtype=wl.FP8_E4M3, block_size=bs)
+        _run(oracle, W, F32, window=100, alibi=True)
+        _run(oracle, W, F32)

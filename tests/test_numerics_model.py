@@ -19,9 +19,16 @@ def _bf16(x):
     return r.view(np.float32)
 
 
-def model_row(q, K, V, scale, split=True, tile=128, gap=8.0):
+def _bf16_trunc(x):
+    """float32 -> bfloat16 by dropping the low 16 bits (toward zero)."""
+    u = np.ascontiguousarray(x, np.float32).view(np.uint32)
+    return (u & np.uint32(0xFFFF0000)).view(np.float32)
+
+
+def model_row(q, K, V, scale, split=True, tile=128, gap=8.0, trunc=False):
     """One query row over keys K [L, D], values V [L, D] (fp32 arrays holding
-    16-bit values), as the chunk kernel computes it."""
+    16-bit values), as the chunk kernel computes it.  trunc: hi and lo are
+    truncations (the bf16 chunk kernel's packing), else nearest even."""
     c = np.float32(scale * LOG2E)
     m = -np.inf
     o = np.zeros(V.shape[1], np.float32)
@@ -36,8 +43,9 @@ def model_row(q, K, V, scale, split=True, tile=128, gap=8.0):
             m = m_tile
         p = np.exp2((s * c - np.float32(m)).astype(np.float32)).astype(np.float32)
         l = np.float32(l + p.sum(dtype=np.float32))
-        hi = _bf16(p)
-        pv = hi if not split else hi + _bf16(p - hi)
+        cut = _bf16_trunc if trunc else _bf16
+        hi = cut(p)
+        pv = hi if not split else hi + cut((p - hi).astype(np.float32))
         o = (o + (pv.astype(np.float64) @ V[j0:j0 + tile].astype(np.float64))).astype(np.float32)
     return o / l
 
@@ -52,8 +60,9 @@ def _bf16_normal(rng, shape, sigma=1.0):
     return _bf16((rng.standard_normal(shape) * sigma).astype(np.float32))
 
 
+@pytest.mark.parametrize("trunc", [False, True])
 @pytest.mark.parametrize("tile", [64, 128])
-def test_hi_lo_split_stays_far_inside_the_bound(tile):
+def test_hi_lo_split_stays_far_inside_the_bound(tile, trunc):
     rng = np.random.default_rng(11)
     D = 128
     scale = D ** -0.5
@@ -61,7 +70,8 @@ def test_hi_lo_split_stays_far_inside_the_bound(tile):
     for L in (1, 2, 3, 17, 64, 65, 128, 129, 700, 2000):
         K, V = _bf16_normal(rng, (L, D)), _bf16_normal(rng, (L, D))
         q = _bf16_normal(rng, D)
-        err = np.abs(model_row(q, K, V, scale, tile=tile) - exact_row(q, K, V, scale)).max()
+        err = np.abs(model_row(q, K, V, scale, tile=tile, trunc=trunc) -
+                     exact_row(q, K, V, scale)).max()
         worst = max(worst, err)
     assert worst < 2e-5
 
@@ -95,3 +105,24 @@ def test_single_bf16_p_can_leave_the_bound():
     pair = np.abs(model_row(q, K, V, 1.0, split=True) - exact).max()
     assert pair < 1e-5
     assert one > 2e-3
+
+
+def test_truncated_pair_on_adversarial_rows():
+    """The bf16 chunk kernel packs P as two truncations (hi = p's upper 16
+    bits, lo = (p - hi)'s): p - (hi + lo) < 2^-14 p, so for values of
+    magnitude 4 the row error stays below 2^-14 * 4 = 2.4e-4 whatever the
+    scores.  Random scores over +-4 values and the two-key row above."""
+    rng = np.random.default_rng(13)
+    one = np.array([1.0], np.float32)
+    worst = 0.0
+    for _ in range(200):
+        L = int(rng.integers(2, 300))
+        K = rng.uniform(-9, 0, size=(L, 1)).astype(np.float32)
+        V = np.where(rng.random((L, 1)) < 0.5, -4.0, 4.0).astype(np.float32)
+        err = np.abs(model_row(one, K, V, 1.0, tile=64, trunc=True) - exact_row(one, K, V, 1.0))
+        worst = max(worst, float(err.max()))
+    assert worst < 2.4e-4
+    x = np.float32(np.log(1.0 + 2.0 ** -8 + 2.0 ** -9.5))
+    K = np.array([[0.0], [x]], np.float32)
+    V = np.array([[-4.0], [4.0]], np.float32)
+    assert np.abs(model_row(one, K, V, 1.0, trunc=True) - exact_row(one, K, V, 1.0)).max() < 2e-5
