@@ -22,8 +22,11 @@
 //     group shares every K/V tile it reads; P enters the PV product as a
 //     hi + lo pair of 16-bit values (p = hi + lo to ~2^-17), which for groups
 //     of up to 4 heads fills the otherwise idle half of the N = 8 columns;
+//   * the running max is raised only when a block's maximum passes it by
+//     more than 2^8 (so P <= 256): most blocks skip the rescale of O;
 //   * FP8 E4M3 tiles are widened to f16 in registers (exact), the per-head
-//     scales folded into the logit multiplier and the output.
+//     scales folded into the logit multiplier and the output; P is one f16
+//     value there (the pools' 5e-2 bound).
 #include "pa_device.cuh"
 #include "pa_launch.h"
 
@@ -41,6 +44,7 @@ constexpr int kBlockTokens = 16;
 constexpr int kMaxPartitionBlocks = 128;  // partition_size <= 1024 tokens, blocks >= 8 tokens
 constexpr int kMaxGroup = 128;            // query heads per KV head
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLazyRaise = 8.f;         // raise the running max when passed by 2^8
 
 enum { KV_F16 = 0, KV_BF16 = 1, KV_FP8 = 2 };
 
@@ -108,6 +112,7 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
   using G = Geo<KVT, D>;
   using S = Smem<KVT, D, GT, NSTAGE>;
   constexpr int kNT = S::kNT;
+  constexpr int kNTPV = kFP8 ? 1 : kNT;   // n-tiles holding P (E4M3 pools: hi only)
   constexpr int kKSteps = D / 16;
   constexpr int kMTiles = D / 16;
   constexpr int kTB = G::kTileBytes;
@@ -167,6 +172,11 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
   const int32_t* bt = a.block_tables + static_cast<int64_t>(seq) * a.max_blocks_per_seq +
                       tok0 / bs;
   for (int i = threadIdx.x; i < npblk; i += kThreads) tbl[i] = bt[i];
+  if constexpr (kFP8) {
+    // one f16 P: the lo columns of P^T are never written and stay zero
+    uint32_t* z = reinterpret_cast<uint32_t*>(pt_all);
+    for (int i = threadIdx.x; i < S::kPT / 4; i += kThreads) z[i] = 0;
+  }
   if (threadIdx.x == 0) {
     for (int i = 0; i < kWarps * NSTAGE; ++i) mbar_init(&bars[i], 1);
     fence_barrier_init();
@@ -360,22 +370,36 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
                           alibi[e & 1] * static_cast<float>(key_base + trel)
                     : -INFINITY;
       }
-      float alpha[2], pv[4];
+      // the running max is raised (and O, l rescaled) only when a block's
+      // maximum passes it by more than 2^8, so P <= 256 and most blocks skip
+      // the rescale (the decision is warp-uniform)
+      float bmx[2];
+      bool need = false;
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         float bm = fmaxf(sv[j], sv[j + 2]);
         bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
         bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
         bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
-        const float m_new = fmaxf(m_run[j], bm);
-        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-        alpha[j] = fast_exp2(m_run[j] - m_use);
+        bmx[j] = bm;
+        need |= bm > m_run[j] + kLazyRaise;
+      }
+      const bool raise = __any_sync(0xffffffffu, need);
+      float alpha[2] = {1.f, 1.f}, pv[4];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        if (raise) {
+          const float m_new = fmaxf(m_run[j], bmx[j]);
+          alpha[j] = fast_exp2(m_run[j] - ((m_new == -INFINITY) ? 0.f : m_new));
+          m_run[j] = m_new;
+        }
+        const float m_use = (m_run[j] == -INFINITY) ? 0.f : m_run[j];
         pv[j] = fast_exp2(sv[j] - m_use);
         pv[j + 2] = fast_exp2(sv[j + 2] - m_use);
         l_run[j] = l_run[j] * alpha[j] + pv[j] + pv[j + 2];
-        m_run[j] = m_new;
       }
-      // ---- P^T (hi, lo) to shared memory: pt[col][token]
+      // ---- P^T (hi, lo) to shared memory: pt[col][token].  E4M3 pools
+      // (5e-2 bound) take one f16 P; their lo columns stay zero.
       const bool writer = (kNT == 2) || (c < 2);
       if (writer) {
 #pragma unroll
@@ -383,48 +407,54 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
           const int t = r + ((e >> 1) << 3);
           const int col = 2 * c + (e & 1);
           const float p = pv[e];
-          uint16_t hi, lo;
-          if constexpr (kMmaBF16) {
-            const __nv_bfloat16 hb = __float2bfloat16_rn(p);
-            hi = __bfloat16_as_ushort(hb);
-            lo = __bfloat16_as_ushort(__float2bfloat16_rn(p - __bfloat162float(hb)));
+          if constexpr (kFP8) {
+            pt[col * kBlockTokens + t] = __half_as_ushort(__float2half_rn(p));
           } else {
-            const __half hh = __float2half_rn(p);
-            hi = __half_as_ushort(hh);
-            lo = __half_as_ushort(__float2half_rn(p - __half2float(hh)));
+            uint16_t hi, lo;
+            if constexpr (kMmaBF16) {
+              const __nv_bfloat16 hb = __float2bfloat16_rn(p);
+              hi = __bfloat16_as_ushort(hb);
+              lo = __bfloat16_as_ushort(__float2bfloat16_rn(p - __bfloat162float(hb)));
+            } else {
+              const __half hh = __float2half_rn(p);
+              hi = __half_as_ushort(hh);
+              lo = __half_as_ushort(__float2half_rn(p - __half2float(hh)));
+            }
+            const int lo_col = (kNT == 2) ? col + 8 : col + 4;
+            pt[col * kBlockTokens + t] = hi;
+            pt[lo_col * kBlockTokens + t] = lo;
           }
-          const int lo_col = (kNT == 2) ? col + 8 : col + 4;
-          pt[col * kBlockTokens + t] = hi;
-          pt[lo_col * kBlockTokens + t] = lo;
         }
       }
       __syncwarp();
       const uint32_t* pt32 = reinterpret_cast<const uint32_t*>(pt);
       uint32_t pb[kNT][2];
 #pragma unroll
-      for (int nt = 0; nt < kNT; ++nt) {
+      for (int nt = 0; nt < kNTPV; ++nt) {
         pb[nt][0] = pt32[(nt * 8 + r) * 8 + c];
         pb[nt][1] = pt32[(nt * 8 + r) * 8 + 4 + c];
       }
-      // ---- rescale the running output, then O^T += V^T P^T
-      float al0 = alpha[0], al1 = alpha[1];
-      if constexpr (kNT == 1) {
-        const float o0 = __shfl_xor_sync(0xffffffffu, al0, 2);
-        const float o1 = __shfl_xor_sync(0xffffffffu, al1, 2);
-        if (c >= 2) {
-          al0 = o0;
-          al1 = o1;
+      // ---- rescale the running output (when raised), then O^T += V^T P^T
+      if (raise) {
+        float al0 = alpha[0], al1 = alpha[1];
+        if constexpr (kNT == 1) {
+          const float o0 = __shfl_xor_sync(0xffffffffu, al0, 2);
+          const float o1 = __shfl_xor_sync(0xffffffffu, al1, 2);
+          if (c >= 2) {
+            al0 = o0;
+            al1 = o1;
+          }
         }
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+          for (int mt = 0; mt < kMTiles; ++mt) {
+            acc[nt][mt][0] *= al0;
+            acc[nt][mt][1] *= al1;
+            acc[nt][mt][2] *= al0;
+            acc[nt][mt][3] *= al1;
+          }
       }
-#pragma unroll
-      for (int nt = 0; nt < kNT; ++nt)
-#pragma unroll
-        for (int mt = 0; mt < kMTiles; ++mt) {
-          acc[nt][mt][0] *= al0;
-          acc[nt][mt][1] *= al1;
-          acc[nt][mt][2] *= al0;
-          acc[nt][mt][3] *= al1;
-        }
       if constexpr (!kFP8) {
         const int mi = lane >> 3, rr = lane & 7;
         const int t = rr + ((mi >> 1) << 3);
@@ -459,7 +489,7 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
           const uint32_t a0 = e4m3x2_to_f16x2(lo01), a1 = e4m3x2_to_f16x2(lo01 >> 16);
           const uint32_t a2 = e4m3x2_to_f16x2(lo23), a3 = e4m3x2_to_f16x2(lo23 >> 16);
 #pragma unroll
-          for (int nt = 0; nt < kNT; ++nt)
+          for (int nt = 0; nt < kNTPV; ++nt)
             mma16816<false>(acc[nt][t], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
         }
       } else {
@@ -483,7 +513,7 @@ paged_attn_kernel(const __grid_constant__ AttnArgs a, const __grid_constant__ CU
             const uint32_t a0 = e4m3x2_to_f16x2(lo01), a1 = e4m3x2_to_f16x2(lo01 >> 16);
             const uint32_t a2 = e4m3x2_to_f16x2(lo23), a3 = e4m3x2_to_f16x2(lo23 >> 16);
 #pragma unroll
-            for (int nt = 0; nt < kNT; ++nt)
+            for (int nt = 0; nt < kNTPV; ++nt)
               mma16816<false>(acc[nt][box * 8 + mm], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
           }
         }
