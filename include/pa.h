@@ -222,8 +222,10 @@ size_t pa_varlen_workspace_size_ex(int32_t num_seqs, int32_t total_q, int32_t nu
  *                cu[num_seqs] = total_q.
  * seqlens_k    : device int32 [num_seqs], kv_len_r >= q_len_r.
  * max_q_len, max_context_len: host upper bounds of q_len_r and kv_len_r (a
- *                request whose kv_len_r exceeds max_context_len is cut there
- *                and reported in the device error word, as for pa_decode).
+ *                request whose kv_len_r exceeds max_context_len is cut there;
+ *                rows run by the decode kernel also report it in the device
+ *                error word, as for pa_decode, but a request of q_len_r >= 2
+ *                taken by the chunk kernel is cut without a report).
  * block_tables : device int32 [num_seqs][max_blocks_per_seq].
  * workspace    : device scratch of at least pa_varlen_workspace_size(...)
  *                bytes (or pa_varlen_workspace_size_ex(...) for these exact
