@@ -62,7 +62,8 @@ typedef enum {
     PA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned buffer */
     PA_ERR_UNSUPPORTED = 2,   /* dtype / head_dim / block_size / group size not built */
     PA_ERR_WORKSPACE = 3,     /* workspace smaller than the *_workspace_size figure */
-    PA_ERR_OUT_OF_RANGE = 4,  /* a kernel met a block id or slot outside the pool */
+    PA_ERR_OUT_OF_RANGE = 4,  /* a kernel met a block id or slot outside the pool, or a
+                                 length above the max_context_len it was promised */
     PA_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed */
     PA_ERR_TIMEOUT = 6        /* a kernel's bounded wait for its own copies expired */
 } pa_status;

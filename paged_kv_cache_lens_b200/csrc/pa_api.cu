@@ -262,7 +262,7 @@ const char* pa_status_string(pa_status status) {
     case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG: invalid argument";
     case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED: configuration not supported";
     case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE: workspace too small";
-    case PA_ERR_OUT_OF_RANGE: return "PA_ERR_OUT_OF_RANGE: block id or slot outside the pool";
+    case PA_ERR_OUT_OF_RANGE: return "PA_ERR_OUT_OF_RANGE: block id or slot outside the pool, or length above max_context_len";
     case PA_ERR_CUDA: return "PA_ERR_CUDA: CUDA runtime or launch failure";
     case PA_ERR_TIMEOUT: return "PA_ERR_TIMEOUT: a kernel gave up a bounded wait";
   }
