@@ -2,13 +2,15 @@
 
 Every function here has the name of the C entry point it calls and does no
 arithmetic of its own: it turns torch tensors into device pointers, sizes and
-dtype codes, passes the current CUDA stream, and raises :class:`PaError` on a
-non-zero status.  The library must be built in-tree
+dtype codes, runs the call on the one device its tensors sit on with that
+device's current CUDA stream (or the stream given), and raises
+:class:`PaError` on a non-zero status.  The library must be built in-tree
 (``python -m paged_kv_cache_lens_b200.build``); importing this module without
 it raises, so there is no silent CPU fallback.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import re
@@ -145,10 +147,36 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream) -> ctypes.c_void_p:
+def _device_of(*tensors) -> Optional[torch.device]:
+    """The one CUDA device the call's device tensors sit on (None and pinned
+    host tensors are skipped; None when no tensor is on a device).  The
+    library launches on the current device and dereferences every pointer
+    there, so tensors on two devices are refused before the call."""
+    dev = None
+    for t in tensors:
+        if t is None or t.device.type != "cuda":
+            continue
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"tensors on {dev} and {t.device}: a call takes one CUDA device")
+    return dev
+
+
+def _on(dev: Optional[torch.device]):
+    """Make `dev` the current device for the call (nothing to do for None)."""
+    return torch.cuda.device(dev) if dev is not None else contextlib.nullcontext()
+
+
+def _stream(stream, dev: Optional[torch.device] = None) -> ctypes.c_void_p:
+    """The stream handle: the given stream, else the current stream of `dev`
+    (of the current device when `dev` is None).  A torch stream of another
+    device than the tensors' is refused."""
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(dev)
     if isinstance(stream, torch.cuda.Stream):
+        if dev is not None and stream.device != dev:
+            raise ValueError(f"stream of {stream.device} for tensors on {dev}")
         return ctypes.c_void_p(stream.cuda_stream)
     return ctypes.c_void_p(int(stream))
 
@@ -190,11 +218,14 @@ def pa_reshape_and_cache(key: torch.Tensor, value: torch.Tensor, slot_mapping: t
     _need(v_cache, "v_cache")
     _need(k_scale, "k_scale", torch.float32)
     _need(v_scale, "v_scale", torch.float32)
+    dev = _device_of(key, value, slot_mapping, k_cache, v_cache, k_scale, v_scale)
     T = key.shape[0]
     desc = cache_desc(k_cache, k_scale, v_scale)
-    st = load_library().pa_reshape_and_cache(
-        _ptr(key), _ptr(value), dtype_code(key.dtype), T, key.stride(0) if T else 0,
-        _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache), ctypes.byref(desc), _stream(stream))
+    with _on(dev):
+        st = load_library().pa_reshape_and_cache(
+            _ptr(key), _ptr(value), dtype_code(key.dtype), T, key.stride(0) if T else 0,
+            _ptr(slot_mapping), _ptr(k_cache), _ptr(v_cache), ctypes.byref(desc),
+            _stream(stream, dev))
     _check(st, "pa_reshape_and_cache")
 
 
@@ -249,6 +280,8 @@ def pa_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache
     _need(context_lens, "context_lens", torch.int32)
     for t, n in ((k_scale, "k_scale"), (v_scale, "v_scale"), (alibi_slopes, "alibi_slopes")):
         _need(t, n, torch.float32)
+    dev = _device_of(out, q, k_cache, v_cache, workspace, block_tables, context_lens, k_scale,
+                     v_scale, alibi_slopes)
     B, hq, d = q.shape
     lib = load_library()
     need = lib.pa_decode_workspace_size(B, hq, d, max_context_len, partition_size)
@@ -259,12 +292,12 @@ def pa_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache
             block_tables.shape[1], _ptr(context_lens), int(max_context_len), float(scale),
             int(partition_size))
     opts = _options(window, alibi_slopes)
-    if opts is None:
-        st = lib.pa_decode(*args, _ptr(workspace), wbytes, _stream(stream))
-        _check(st, "pa_decode")
-    else:
-        st = lib.pa_decode_ex(*args, opts, _ptr(workspace), wbytes, _stream(stream))
-        _check(st, "pa_decode_ex")
+    with _on(dev):
+        if opts is None:
+            st = lib.pa_decode(*args, _ptr(workspace), wbytes, _stream(stream, dev))
+        else:
+            st = lib.pa_decode_ex(*args, opts, _ptr(workspace), wbytes, _stream(stream, dev))
+    _check(st, "pa_decode" if opts is None else "pa_decode_ex")
 
 
 def pa_varlen(out: torch.Tensor, q: torch.Tensor, cu_seqlens_q: torch.Tensor,
@@ -282,6 +315,8 @@ def pa_varlen(out: torch.Tensor, q: torch.Tensor, cu_seqlens_q: torch.Tensor,
         _need(t, n, torch.int32)
     for t, n in ((k_scale, "k_scale"), (v_scale, "v_scale"), (alibi_slopes, "alibi_slopes")):
         _need(t, n, torch.float32)
+    dev = _device_of(out, q, k_cache, v_cache, workspace, cu_seqlens_q, seqlens_k, block_tables,
+                     k_scale, v_scale, alibi_slopes)
     total_q, hq, d = q.shape
     S = seqlens_k.shape[0]
     lib = load_library()
@@ -297,12 +332,12 @@ def pa_varlen(out: torch.Tensor, q: torch.Tensor, cu_seqlens_q: torch.Tensor,
             _ptr(k_cache), _ptr(v_cache), ctypes.byref(desc), _ptr(block_tables),
             block_tables.shape[1], float(scale))
     opts = _options(window, alibi_slopes)
-    if opts is None:
-        st = lib.pa_varlen(*args, _ptr(workspace), wbytes, _stream(stream))
-        _check(st, "pa_varlen")
-    else:
-        st = lib.pa_varlen_ex(*args, opts, _ptr(workspace), wbytes, _stream(stream))
-        _check(st, "pa_varlen_ex")
+    with _on(dev):
+        if opts is None:
+            st = lib.pa_varlen(*args, _ptr(workspace), wbytes, _stream(stream, dev))
+        else:
+            st = lib.pa_varlen_ex(*args, opts, _ptr(workspace), wbytes, _stream(stream, dev))
+    _check(st, "pa_varlen" if opts is None else "pa_varlen_ex")
 
 
 def pa_hbm_read_probe(buf: torch.Tensor, sink: torch.Tensor, stream=None) -> None:
@@ -310,8 +345,10 @@ def pa_hbm_read_probe(buf: torch.Tensor, sink: torch.Tensor, stream=None) -> Non
     device int32 of one element) receives the XOR of its 32-bit words."""
     _need(buf, "buf")
     _need(sink, "sink")
-    st = load_library().pa_hbm_read_probe(_ptr(buf), buf.numel() * buf.element_size(),
-                                          _ptr(sink), _stream(stream))
+    dev = _device_of(buf, sink)
+    with _on(dev):
+        st = load_library().pa_hbm_read_probe(_ptr(buf), buf.numel() * buf.element_size(),
+                                              _ptr(sink), _stream(stream, dev))
     _check(st, "pa_hbm_read_probe")
 
 
@@ -332,10 +369,12 @@ def pa_copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, block_mapping: 
     _need(k_cache, "k_cache")
     _need(v_cache, "v_cache")
     _need(block_mapping, "block_mapping", torch.int64)
+    dev = _device_of(k_cache, v_cache, block_mapping)
     desc = cache_desc(k_cache)
     n = block_mapping.shape[0]
-    st = load_library().pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), ctypes.byref(desc),
-                                       _ptr(block_mapping), n, _stream(stream))
+    with _on(dev):
+        st = load_library().pa_copy_blocks(_ptr(k_cache), _ptr(v_cache), ctypes.byref(desc),
+                                           _ptr(block_mapping), n, _stream(stream, dev))
     _check(st, "pa_copy_blocks")
 
 
@@ -346,9 +385,12 @@ def pa_swap_blocks(dst_k: torch.Tensor, dst_v: torch.Tensor, src_k: torch.Tensor
     import numpy as np
     for t, n in ((dst_k, "dst_k"), (dst_v, "dst_v"), (src_k, "src_k"), (src_v, "src_v")):
         _need(t, n, pinned_ok=True)
+    dev = _device_of(dst_k, dst_v, src_k, src_v)
     pairs = np.ascontiguousarray(np.asarray(block_mapping, dtype=np.int64).reshape(-1, 2))
     desc = cache_desc(src_k)
-    st = load_library().pa_swap_blocks(
-        _ptr(dst_k), _ptr(dst_v), _ptr(src_k), _ptr(src_v), ctypes.byref(desc), src_k.shape[0],
-        dst_k.shape[0], ctypes.c_void_p(pairs.ctypes.data), len(pairs), _stream(stream))
+    with _on(dev):
+        st = load_library().pa_swap_blocks(
+            _ptr(dst_k), _ptr(dst_v), _ptr(src_k), _ptr(src_v), ctypes.byref(desc),
+            src_k.shape[0], dst_k.shape[0], ctypes.c_void_p(pairs.ctypes.data), len(pairs),
+            _stream(stream, dev))
     _check(st, "pa_swap_blocks")

@@ -57,3 +57,111 @@ def test_layout_and_dtype_checks():
     with pytest.raises(ValueError, match="contiguous"):   # a strided view where none is allowed
         need(k, "k_cache")
     need(None, "absent")                                  # optional arguments pass
+
+
+class _DevTensor:
+    """Stands in for a CUDA tensor on a host without a GPU: the attributes the
+    binding reads (device, shape, dtype, strides, pointer)."""
+
+    def __init__(self, shape, dtype, device):
+        self.shape = torch.Size(shape)
+        self.dtype = dtype
+        self.device = torch.device(device)
+        self._ptr = 0x10000 * (1 + len(shape))
+
+    def data_ptr(self):
+        return self._ptr
+
+    def stride(self, dim=None):
+        s = torch.empty(self.shape, device="meta").stride()
+        return s if dim is None else s[dim]
+
+    def numel(self):
+        return self.shape.numel()
+
+    def element_size(self):
+        return torch.empty((), dtype=self.dtype, device="meta").element_size()
+
+
+class _FakeLib:
+    def __init__(self):
+        self.calls = []
+
+    def __getattr__(self, name):
+        def call(*args):
+            self.calls.append(name)
+            return 0
+        return call
+
+
+def _fake_cuda(monkeypatch):
+    """The binding with its tensor checks, library and device switch replaced
+    by recorders; returns (library, list of devices made current, list of
+    devices whose current stream was taken)."""
+    lib, entered, streams = _FakeLib(), [], []
+    monkeypatch.setattr(pa, "_need", lambda *a, **k: None)
+    monkeypatch.setattr(pa, "load_library", lambda *a, **k: lib)
+
+    class _Dev:
+        def __init__(self, d):
+            self.d = d
+
+        def __enter__(self):
+            entered.append(self.d)
+
+        def __exit__(self, *exc):
+            return False
+
+    monkeypatch.setattr(torch.cuda, "device", _Dev)
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda d=None: streams.append(d) or 0)
+    return lib, entered, streams
+
+
+def test_each_call_runs_on_its_tensors_device(monkeypatch):
+    """Every entry point makes the device of its tensors current for the call
+    and takes that device's stream, not the current device's."""
+    lib, entered, streams = _fake_cuda(monkeypatch)
+    d1 = torch.device("cuda", 1)
+    T = lambda *s, dt=torch.bfloat16: _DevTensor(s, dt, d1)  # noqa: E731
+    kc, vc = T(8, 2, 16, 64), T(8, 2, 16, 64)
+    i32 = torch.int32
+    pa.pa_reshape_and_cache(T(2, 2, 64), T(2, 2, 64), T(2, dt=torch.int64), kc, vc)
+    pa.pa_decode(T(2, 4, 64), T(2, 4, 64), kc, vc, T(2, 4, dt=i32), T(2, dt=i32), 16, 0.125)
+    pa.pa_decode(T(2, 4, 64), T(2, 4, 64), kc, vc, T(2, 4, dt=i32), T(2, dt=i32), 16, 0.125,
+                 window=8)
+    pa.pa_varlen(T(3, 4, 64), T(3, 4, 64), T(3, dt=i32), T(2, dt=i32), 2, 16, kc, vc,
+                 T(2, 4, dt=i32), 0.125)
+    pa.pa_varlen(T(3, 4, 64), T(3, 4, 64), T(3, dt=i32), T(2, dt=i32), 2, 16, kc, vc,
+                 T(2, 4, dt=i32), 0.125, alibi_slopes=T(4, dt=torch.float32))
+    pa.pa_copy_blocks(kc, vc, T(1, 2, dt=torch.int64))
+    pa.pa_hbm_read_probe(T(64, dt=i32), T(1, dt=i32))
+    host = _DevTensor((8, 2, 16, 64), torch.bfloat16, "cpu")        # a pinned host pool
+    pa.pa_swap_blocks(host, host, kc, vc, np.zeros((1, 2), np.int64))
+    launched = [c for c in lib.calls if "workspace" not in c]
+    assert launched == ["pa_reshape_and_cache", "pa_decode", "pa_decode_ex", "pa_varlen",
+                        "pa_varlen_ex", "pa_copy_blocks", "pa_hbm_read_probe", "pa_swap_blocks"]
+    assert entered == [d1] * len(launched)
+    assert streams == [d1] * len(launched)
+
+
+def test_tensors_on_two_devices_are_refused(monkeypatch):
+    lib, entered, _ = _fake_cuda(monkeypatch)
+    a = lambda *s, dt=torch.bfloat16: _DevTensor(s, dt, "cuda:0")  # noqa: E731
+    b = lambda *s, dt=torch.bfloat16: _DevTensor(s, dt, "cuda:1")  # noqa: E731
+    i32 = torch.int32
+    with pytest.raises(ValueError, match="one CUDA device"):
+        pa.pa_decode(a(2, 4, 64), a(2, 4, 64), b(8, 2, 16, 64), b(8, 2, 16, 64), a(2, 4, dt=i32),
+                     a(2, dt=i32), 16, 0.125)
+    with pytest.raises(ValueError, match="one CUDA device"):
+        pa.pa_copy_blocks(a(8, 2, 16, 64), a(8, 2, 16, 64), b(1, 2, dt=torch.int64))
+    with pytest.raises(ValueError, match="one CUDA device"):
+        pa.pa_swap_blocks(a(8, 2, 16, 64), a(8, 2, 16, 64), b(8, 2, 16, 64), b(8, 2, 16, 64),
+                          np.zeros((1, 2), np.int64))
+    assert lib.calls == [] and entered == []
+
+
+def test_device_of_skips_host_and_absent_tensors():
+    host = _DevTensor((4,), torch.float32, "cpu")
+    dev = _DevTensor((4,), torch.float32, "cuda:3")
+    assert pa._device_of(None, host) is None
+    assert pa._device_of(host, None, dev, dev) == torch.device("cuda", 3)
