@@ -454,19 +454,19 @@ int oracle_paged_attention_ex(double *out, double *lse, const void *q, int q_dty
     if (nt == 1) {
         attn_worker(&slices[0]);
     } else {
-        int started = 0;
+        /* a slice whose thread could not be started runs here instead;
+           started[w] says which threads there are to join */
+        unsigned char *started = (unsigned char *)calloc((size_t)nt, 1);
         for (int w = 0; w < nt; ++w) {
-            if (pthread_create(&tids[w], NULL, attn_worker, &slices[w]) != 0) {
-                attn_worker(&slices[w]);       /* run it here instead */
-                tids[w] = 0;
-            } else {
-                started++;
-            }
+            if (started && pthread_create(&tids[w], NULL, attn_worker, &slices[w]) == 0)
+                started[w] = 1;
+            else
+                attn_worker(&slices[w]);
         }
         for (int w = 0; w < nt; ++w)
-            if (tids[w])
+            if (started && started[w])
                 pthread_join(tids[w], NULL);
-        (void)started;
+        free(started);
     }
     free(slices);
     free(tids);
