@@ -73,3 +73,72 @@ def test_oracle_copy_blocks(oracle):
     assert np.array_equal(hk[:2], kc[3:5]) and np.array_equal(hv[:2], vc[3:5])
     with pytest.raises(ValueError):
         oracle.copy_blocks(hk, hv, kc, vc, [[3, 4]])
+
+
+def test_a_table_that_does_not_fit_takes_no_block():
+    bm = BlockManager(3)
+    bm.allocate_table(20)                             # 2 blocks
+    with pytest.raises(OutOfBlocks):
+        bm.allocate_table(40)                         # 3 needed, 1 free
+    assert list(bm.free) == [2] and bm.ref_count(2) == 0
+
+
+def test_misuse_is_refused_with_the_counts_unchanged():
+    bm = BlockManager(8)
+    t = bm.allocate_table(40)                         # blocks 0, 1, 2
+    with pytest.raises(ValueError):
+        bm.release(5)                                 # never allocated
+    with pytest.raises(ValueError):
+        bm.fork(t, 0)
+    with pytest.raises(ValueError):
+        bm.fork(t + [6], 2)                           # block 6 is not held
+    with pytest.raises(ValueError):
+        bm.free_table([0, 0, 1])                      # block 0 held once, listed twice
+    assert [bm.ref_count(b) for b in range(8)] == [1, 1, 1, 0, 0, 0, 0, 0]
+    with pytest.raises(ValueError):
+        bm.append_slot(t, 49)                         # the sequence holds at most 48 tokens
+    with pytest.raises(ValueError):
+        bm.append_slot(t, -1)
+    assert t == [0, 1, 2] and len(bm.free) == 5
+    slot, copy = bm.append_slot(t, 48)                # the next token opens block 3
+    assert copy is None and t == [0, 1, 2, 3] and slot == 48
+
+
+@pytest.mark.parametrize("order", [[0, 1, 1], [0, 5], [-1, 2]])
+def test_free_order_must_name_distinct_pool_blocks(order):
+    with pytest.raises(ValueError):
+        BlockManager(4, free_order=order)
+
+
+def test_random_fork_append_free_keeps_the_pool_consistent():
+    """Seeded random traffic of new sequences, forks, appends (with their
+    copy-on-write) and frees: at every step each block is either free or held,
+    never both, and its count equals the number of table entries naming it."""
+    rng = np.random.default_rng(5)
+    bm = BlockManager(64, block_size=4)
+    seqs = []                                         # [table, tokens]
+    for _ in range(3000):
+        op = rng.integers(4)
+        try:
+            if op == 0 or not seqs:
+                n = int(rng.integers(0, 13))
+                seqs.append([bm.allocate_table(n), n])
+            elif op == 1:
+                i = int(rng.integers(len(seqs)))
+                for t in bm.fork(seqs[i][0], int(rng.integers(1, 4)))[1:]:
+                    seqs.append([t, seqs[i][1]])
+            elif op == 2:
+                s = seqs[int(rng.integers(len(seqs)))]
+                bm.append_slot(s[0], s[1])
+                s[1] += 1
+            else:
+                bm.free_table(seqs.pop(int(rng.integers(len(seqs))))[0])
+        except OutOfBlocks:
+            pass
+        held = {}
+        for t, n in seqs:
+            assert len(t) == -(-n // 4)
+            for b in t:
+                held[b] = held.get(b, 0) + 1
+        assert held == bm.ref
+        assert not set(bm.free) & set(held) and len(bm.free) + len(held) == 64
