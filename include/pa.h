@@ -37,7 +37,9 @@
  *   - Block-table entries at or past ceil(len / block_size) are never read.
  *     Entries that are read and fall outside [0, num_blocks) are skipped
  *     (treated as masked) and recorded in the device error word.
- *   - GQA: query head hq reads KV head hq / (num_q_heads / num_kv_heads).
+ *   - GQA: query head hq reads KV head hq / (num_q_heads / num_kv_heads);
+ *     num_q_heads is a multiple of num_kv_heads, the group at most 128 (MHA,
+ *     GQA and MQA alike).
  *   - Attention accumulates in fp32; softmax is exact up to rounding.
  */
 #ifndef PA_H_
@@ -72,9 +74,9 @@ typedef enum {
  * are device pointers). */
 typedef struct {
     int32_t num_blocks;     /* physical blocks in the pool */
-    int32_t block_size;     /* tokens per block: 16 */
+    int32_t block_size;     /* tokens per block: 8, 16 or 32 */
     int32_t num_kv_heads;
-    int32_t head_dim;       /* 64, 128 or 256 (FP8: 128 or 256) */
+    int32_t head_dim;       /* 64, 128 or 256, for every kv_dtype */
     pa_dtype kv_dtype;      /* PA_F16, PA_BF16 or PA_FP8_E4M3 */
     const float* k_scale;   /* [num_kv_heads] device fp32, FP8 only, else NULL */
     const float* v_scale;   /* [num_kv_heads] device fp32, FP8 only, else NULL */
@@ -213,10 +215,11 @@ size_t pa_varlen_workspace_size_ex(int32_t num_seqs, int32_t total_q, int32_t nu
  * kv_len_r - q_len_r + i and attends keys 0 .. kv_len_r - q_len_r + i
  * (causal mask aligned to the bottom right).  Rows with no visible key yield
  * zeros.  q_len 1 rows are decode rows; longer ones are prefill chunks.
- * Chunks run on the tensor-core chunk kernel when the pool is bf16/f16 with
- * head_dim 64, 128 or 256, q has the pool's type, the GQA group is a power
- * of two up to 128 and out is 16-byte aligned; otherwise every row runs on
- * the decode kernel.  Either way the result is the same attention.
+ * Chunks run on the tensor-core chunk kernel when the GQA group is a power
+ * of two up to 128, out is 16-byte aligned, and either the pool is bf16/f16
+ * with head_dim 64, 128 or 256 and q of the pool's type, or the pool is
+ * E4M3 with head_dim 128 and q f16 or bf16; otherwise every row runs on the
+ * decode kernel.  Either way the result is the same attention.
  *
  * out, q       : device [total_q][num_q_heads][head_dim].
  * cu_seqlens_q : device int32 [num_seqs + 1], non-decreasing, cu[0] = 0,
