@@ -356,7 +356,8 @@ pa_status pa_selftest_wait_timeout(void* stream);
  * Read and clear the device error word that kernels set when they skip an
  * out-of-range block id or slot, or cut a row whose context_lens / seqlens_k
  * entry exceeds the max_context_len it was promised (PA_ERR_OUT_OF_RANGE; the
- * row's attention then covers its first max_context_len keys only), or give
+ * row's attention then covers its first max_context_len keys only; rows of a
+ * pa_varlen chunk on the tensor-core path are cut without a report), or give
  * up a bounded wait (PA_ERR_TIMEOUT).  Synchronises `stream` first.  Returns PA_OK when no
  * kernel reported anything since the last call.
  */
