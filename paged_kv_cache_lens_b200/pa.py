@@ -27,7 +27,6 @@ PA_OK = 0
 STATUS_NAMES = {0: "PA_OK", 1: "PA_ERR_INVALID_ARG", 2: "PA_ERR_UNSUPPORTED",
                 3: "PA_ERR_WORKSPACE", 4: "PA_ERR_OUT_OF_RANGE", 5: "PA_ERR_CUDA",
                 6: "PA_ERR_TIMEOUT"}
-BLOCK_SIZE = 16
 
 
 class PaError(RuntimeError):
@@ -208,7 +207,7 @@ def pa_reshape_and_cache(key: torch.Tensor, value: torch.Tensor, slot_mapping: t
                          k_cache: torch.Tensor, v_cache: torch.Tensor, k_scale=None,
                          v_scale=None, stream=None) -> None:
     """key/value: [T, Hkv, D] (rows may be strided, e.g. views into a fused QKV
-    buffer); slot_mapping: int64 [T]; pools [NB, Hkv, 16, D]."""
+    buffer); slot_mapping: int64 [T]; pools [NB, Hkv, block_size, D]."""
     _need(key, "key", rows_strided=True)
     _need(value, "value", rows_strided=True)
     if key.shape != value.shape or key.stride() != value.stride():
