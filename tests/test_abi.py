@@ -2,7 +2,6 @@
 header declares, and answers the host-only calls (status strings, workspace
 sizing, argument validation) without touching a GPU."""
 import ctypes
-import os
 import re
 
 import pytest

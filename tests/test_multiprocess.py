@@ -3,7 +3,6 @@ own replica, reduce to the slowest rank's time; only rank 0 reports."""
 import os
 import socket
 
-import pytest
 import torch.multiprocessing as mp
 
 

@@ -7,7 +7,6 @@ values leaves it."""
 import numpy as np
 import pytest
 
-from paged_kv_cache_lens_b200 import workloads as wl
 
 LOG2E = 1.4426950408889634
 

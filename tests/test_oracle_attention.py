@@ -10,7 +10,6 @@ independent NumPy twin.
 import math
 
 import numpy as np
-import pytest
 import torch
 
 from oracle import pa_oracle_np as npo
