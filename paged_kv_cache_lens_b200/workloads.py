@@ -38,10 +38,6 @@ def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     return ((u + np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)).astype(np.uint16)
 
 
-def f32_to_f16_bits(x: np.ndarray) -> np.ndarray:
-    return np.asarray(x, dtype=np.float32).astype(np.float16).view(np.uint16)
-
-
 def bits_to_f32(bits: np.ndarray, dtype: int) -> np.ndarray:
     """Widen bf16/f16 bit patterns to fp32 (exact)."""
     if dtype == BF16:
