@@ -10,11 +10,12 @@ independent NumPy twin.
 import math
 
 import numpy as np
+import pytest
 import torch
 
 from oracle import pa_oracle_np as npo
 from paged_kv_cache_lens_b200 import workloads as wl
-from tests._helpers import oracle_attention, oracle_pools
+from tests._helpers import NAN_FILL, oracle_attention, oracle_pools
 
 
 def _f64(bits, dtype):
@@ -276,3 +277,56 @@ def test_never_reads_unwritten_slots(oracle):
     out = oracle_attention(oracle, W, kc, vc)
     assert np.all(np.isfinite(out))
     assert np.isnan(_f64(kc, W.kv_dtype)).any()
+
+
+def _relayout(W, kc, vc, bs, seed):
+    """The same logical K/V of every request, moved byte for byte into a pool
+    of `bs`-token blocks under a fresh seeded random block table (the paging
+    of "PagedAttention 与 Continuous Batching", §3.3: token t of a request
+    lives at table[t / bs] * bs + t % bs, for any block size of §3.7)."""
+    import dataclasses
+    rng = np.random.default_rng(seed)
+    need = [-(-int(L) // bs) for L in W.seqlens_k]
+    nb = max(1, sum(need) + 3)
+    ids = rng.permutation(nb).astype(np.int32)
+    tables = np.full((W.num_seqs, max(need) + 1), -1, np.int32)
+    shape = (nb, W.num_kv_heads, bs, W.head_dim)
+    k2, v2 = np.zeros(shape, kc.dtype), np.zeros(shape, vc.dtype)
+    cur = 0
+    for r, n in enumerate(need):
+        tables[r, :n] = ids[cur:cur + n]
+        cur += n
+        t = np.arange(int(W.seqlens_k[r]))
+        old_b, old_o = W.block_tables[r, t // W.block_size], t % W.block_size
+        new_b, new_o = tables[r, t // bs], t % bs
+        k2[new_b, :, new_o, :] = kc[old_b, :, old_o, :]
+        v2[new_b, :, new_o, :] = vc[old_b, :, old_o, :]
+    W2 = dataclasses.replace(W, block_size=bs, block_tables=tables, num_blocks=nb)
+    return W2, k2, v2
+
+
+@pytest.mark.parametrize("kv", [None, wl.FP8_E4M3])
+@pytest.mark.parametrize("bs", [8, 32])
+def test_block_size_changes_nothing(oracle, bs, kv):
+    """The same logical cache laid out in 8- or 32-token blocks gives bitwise
+    the result of 16-token blocks, and matches float64 SDPA."""
+    W = _small_varlen(seed=41, kv_dtype=kv)
+    kc, vc = oracle_pools(oracle, W)
+    want = oracle_attention(oracle, W, kc, vc)
+    W2, k2, v2 = _relayout(W, kc, vc, bs, seed=42)
+    got = oracle_attention(oracle, W2, k2, v2)
+    assert np.array_equal(got, want)
+    np.testing.assert_allclose(got, _sdpa_reference(W2, k2, v2), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("kv", [None, wl.FP8_E4M3])
+@pytest.mark.parametrize("bs", [8, 32])
+def test_cache_write_at_other_block_sizes_matches_numpy_twin(oracle, bs, kv):
+    W = wl.build_workload("bsw", 43, [1, 9, 1, 3], [20, 9, 70, 41], 4, 2, 16, kv_dtype=kv,
+                          block_size=bs)
+    kc, vc = oracle_pools(oracle, W)
+    kt = np.full_like(kc, NAN_FILL[W.kv_dtype])                 # the oracle pools' fill too
+    vt = np.full_like(vc, NAN_FILL[W.kv_dtype])
+    for k, v, s in ((W.prefill_k, W.prefill_v, W.prefill_slots), (W.new_k, W.new_v, W.new_slots)):
+        npo.reshape_and_cache(k, v, W.src_dtype, s, kt, vt, W.kv_dtype, W.k_scale, W.v_scale)
+    assert np.array_equal(kt, kc) and np.array_equal(vt, vc)

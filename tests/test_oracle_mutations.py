@@ -31,6 +31,9 @@ MUTATIONS = {
     "alibi_sign": ("slope * (double)(t - last)", "slope * (double)(last - t)"),
     "table_row_stride": ("J->block_tables[(int64_t)r * J->max_blocks_per_seq + t / J->block_size]",
                          "J->block_tables[(int64_t)r * (J->max_blocks_per_seq - 1) + t / J->block_size]"),
+    "gather_assumes_16_token_blocks": ("J->block_tables[(int64_t)r * J->max_blocks_per_seq + t / J->block_size]",
+                                       "J->block_tables[(int64_t)r * J->max_blocks_per_seq + t / 16]"),
+    "scatter_assumes_16_token_blocks": ("int64_t blk = slot / block_size;", "int64_t blk = slot / 16;"),
 }
 
 
@@ -41,9 +44,9 @@ def _sdpa(W, kc, vc):
     for r in range(W.num_seqs):
         r0, r1, L = int(W.cu_seqlens_q[r]), int(W.cu_seqlens_q[r + 1]), int(W.seqlens_k[r])
         t = np.arange(L)
-        blk = W.block_tables[r, t // 16]
-        k = npo.to_f64(kc[blk, :, t % 16, :], W.kv_dtype)
-        v = npo.to_f64(vc[blk, :, t % 16, :], W.kv_dtype)
+        blk = W.block_tables[r, t // W.block_size]
+        k = npo.to_f64(kc[blk, :, t % W.block_size, :], W.kv_dtype)
+        v = npo.to_f64(vc[blk, :, t % W.block_size, :], W.kv_dtype)
         if W.kv_dtype == wl.FP8_E4M3:
             k = k * W.k_scale.astype(np.float64)[None, :, None]
             v = v * W.v_scale.astype(np.float64)[None, :, None]
@@ -60,7 +63,8 @@ def _sdpa(W, kc, vc):
 def _pins_pass(orc) -> bool:
     """A compact run of the pins: codec round trip and midpoints, the scatter
     against the NumPy twin, attention against float64 SDPA on a GQA varlen
-    batch with bf16 and FP8 pools."""
+    batch with bf16 and FP8 pools of 16-token blocks and a bf16 pool of
+    8-token blocks."""
     try:
         for b in range(0x7E):
             if orc.e4m3_from_float(orc.e4m3_to_double(b)) != b:
@@ -69,8 +73,9 @@ def _pins_pass(orc) -> bool:
             mid = (lo + hi) / 2
             if float(np.float32(mid)) == mid and orc.e4m3_from_float(mid) != (b if b % 2 == 0 else b + 1):
                 return False
-        for kv in (None, wl.FP8_E4M3):
-            W = wl.build_workload("m", 31, [1, 6, 1, 20], [30, 6, 17, 52], 4, 2, 16, kv_dtype=kv)
+        for kv, bs in ((None, 16), (wl.FP8_E4M3, 16), (None, 8)):
+            W = wl.build_workload("m", 31, [1, 6, 1, 20], [30, 6, 17, 52], 4, 2, 16, kv_dtype=kv,
+                                  block_size=bs)
             kc, vc = oracle_pools(orc, W)
             kt, vt = np.full_like(kc, kc.flat[-1]), np.full_like(vc, vc.flat[-1])
             kt[:], vt[:] = (0x7F if kv else 0x7FC0), (0x7F if kv else 0x7FC0)
