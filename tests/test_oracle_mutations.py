@@ -34,6 +34,10 @@ MUTATIONS = {
     "gather_assumes_16_token_blocks": ("J->block_tables[(int64_t)r * J->max_blocks_per_seq + t / J->block_size]",
                                        "J->block_tables[(int64_t)r * J->max_blocks_per_seq + t / 16]"),
     "scatter_assumes_16_token_blocks": ("int64_t blk = slot / block_size;", "int64_t blk = slot / 16;"),
+    "fp8_dequant_scale_of_head_0": ("*v *= (double)sc[h];", "*v *= (double)sc[0];"),
+    "fp8_quant_scale_of_head_0": ("/ (double)k_scale[h]);", "/ (double)k_scale[0]);"),
+    "query_of_head_0": ("(row * J->num_q_heads + hq) * (int64_t)D + d",
+                        "(row * J->num_q_heads) * (int64_t)D + d"),
 }
 
 
