@@ -38,6 +38,8 @@ MUTATIONS = {
     "fp8_quant_scale_of_head_0": ("/ (double)k_scale[h]);", "/ (double)k_scale[0]);"),
     "query_of_head_0": ("(row * J->num_q_heads + hq) * (int64_t)D + d",
                         "(row * J->num_q_heads) * (int64_t)D + d"),
+    "alibi_slope_of_kv_head": ("(double)J->alibi_slopes[hq]", "(double)J->alibi_slopes[h]"),
+    "window_from_request_end": ("first = last - J->window + 1;", "first = kv_len - J->window;"),
 }
 
 
