@@ -1,6 +1,8 @@
 """The pins catch plausible mistakes: each case plants one mistake in a
 temporary copy of the oracle's C source (on the CPU), rebuilds it, and checks
 that at least one pin fails for the planted copy while the real oracle passes.
+Every planted mistake keeps its reads and writes inside the arrays it is
+given, so a planted copy returns wrong values rather than corrupting memory.
 """
 import os
 
@@ -40,6 +42,10 @@ MUTATIONS = {
                         "(row * J->num_q_heads) * (int64_t)D + d"),
     "alibi_slope_of_kv_head": ("(double)J->alibi_slopes[hq]", "(double)J->alibi_slopes[h]"),
     "window_from_request_end": ("first = last - J->window + 1;", "first = kv_len - J->window;"),
+    "copy_skips_last_pair": ("for (int64_t i = 0; i < num_pairs; ++i)",
+                             "for (int64_t i = 0; i < num_pairs - 1; ++i)"),
+    "copy_half_of_each_k_block": ("(size_t)block_bytes);", "(size_t)block_bytes / 2);"),
+    "copy_v_from_k_pool": ("(const char *)src_v + s * block_bytes,", "(const char *)src_k + s * block_bytes,"),
 }
 
 
@@ -70,7 +76,8 @@ def _pins_pass(orc) -> bool:
     """A compact run of the pins: codec round trip and midpoints, the scatter
     against the NumPy twin, attention against float64 SDPA on a GQA varlen
     batch with bf16 and FP8 pools of 16-token blocks and a bf16 pool of
-    8-token blocks."""
+    8-token blocks, and whole-block copies within a pool and between two pools
+    against plain array assignment."""
     try:
         for b in range(0x7E):
             if orc.e4m3_from_float(orc.e4m3_to_double(b)) != b:
@@ -100,6 +107,19 @@ def _pins_pass(orc) -> bool:
         sl = np.array([0.5, 0.25, 0.125, 0.0625], np.float32)
         got = oracle_attention(orc, W, kc, vc, window=11, alibi_slopes=sl)
         if not np.allclose(got, _reference(W, kc, vc, window=11, slopes=sl), rtol=0, atol=1e-12):
+            return False
+        rng = np.random.default_rng(33)
+        pk = rng.integers(0, 1 << 16, (9, 2, 16, 8)).astype(np.uint16)
+        pv = rng.integers(0, 1 << 16, (9, 2, 16, 8)).astype(np.uint16)
+        hk, hv = np.zeros((5, 2, 16, 8), np.uint16), np.zeros((5, 2, 16, 8), np.uint16)
+        wk, wv = pk.copy(), pv.copy()
+        wk[[6, 0]], wv[[6, 0]] = pk[[2, 5]], pv[[2, 5]]
+        orc.copy_blocks(pk, pv, pk, pv, [[2, 6], [5, 0]])
+        orc.copy_blocks(hk, hv, pk, pv, [[3, 4], [7, 1]])
+        if not (np.array_equal(pk, wk) and np.array_equal(pv, wv)):
+            return False
+        if not (np.array_equal(hk[[4, 1]], wk[[3, 7]]) and np.array_equal(hv[[4, 1]], wv[[3, 7]])
+                and not hk[[0, 2, 3]].any() and not hv[[0, 2, 3]].any()):
             return False
         return True
     except (ValueError, IndexError):
