@@ -21,6 +21,7 @@ and reduced as the max over ranks.
 from __future__ import annotations
 
 import argparse
+import atexit
 import datetime
 import json
 import os
@@ -140,7 +141,9 @@ def workload_name(W) -> str:
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons.  Sampling starts
     before the timed region; summary() keeps the samples stamped inside it
-    (widened by the sampling period, so a short region still gets one)."""
+    (widened by the sampling period, so a short region still gets one).  At
+    interpreter exit a sampler still running (a run that raised before
+    stop()) is killed and the sample file removed."""
 
     PERIOD_MS = 50
 
@@ -150,6 +153,16 @@ class ClockSampler:
         fd, self.path = tempfile.mkstemp(prefix=f"pa_clocks_{device_index}_", suffix=".csv")
         os.close(fd)
         self.t0 = self.t1 = None
+        atexit.register(self._cleanup)
+
+    def _cleanup(self):
+        if self.proc is not None and self.proc.poll() is None:
+            self.proc.kill()
+            self.proc.wait()
+        try:
+            os.unlink(self.path)
+        except OSError:
+            pass
 
     def start(self):
         try:

@@ -11,12 +11,17 @@ import bench
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
+class _Finished:
+    def poll(self):
+        return 0
+
+
 def _summary_of(lines, t0, t1):
     s = bench.ClockSampler(0)
     try:
         with open(s.path, "w") as f:
             f.write("\n".join(lines) + "\n")
-        s.proc = object()                  # stands in for a finished nvidia-smi process
+        s.proc = _Finished()               # stands in for a finished nvidia-smi process
         s.t0, s.t1 = t0, t1
         return s.summary()
     finally:
@@ -74,3 +79,14 @@ def test_reference_arm_prints_one_json_line():
     assert d["impl"] == "reference" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+
+
+def test_sampler_left_running_is_killed_at_exit():
+    """A run that raises between start() and stop() must not leave an endless
+    sampler behind: the exit hook kills it and removes the sample file."""
+    s = bench.ClockSampler(0)
+    s.proc = subprocess.Popen(["sleep", "60"])     # stands in for nvidia-smi -lms
+    assert os.path.exists(s.path) and s.proc.poll() is None
+    s._cleanup()
+    assert s.proc.poll() is not None and not os.path.exists(s.path)
+    s._cleanup()                                   # a second call (the real exit) is harmless
