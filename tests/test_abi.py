@@ -177,3 +177,25 @@ def test_block_ops_and_probe_validation(lib):
     assert lib.pa_hbm_read_probe(fake, -16, fake, None) == 1
     assert lib.pa_hbm_read_probe(fake, 32, None, None) == 1
     assert lib.pa_hbm_read_probe(P(0x10008), 32, fake, None) == 1
+
+
+def test_static_decode_and_varlen_options_validation(lib):
+    """Refusals that come before any CUDA call: pa_decode_static without a
+    pool description or with partials past its fixed scratch, and pa_varlen_ex
+    with ALiBi slopes that are not a 4-byte aligned float array."""
+    P, i32, E, F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int, ctypes.c_float
+    lib.pa_decode_static.argtypes = [P, E, P, E, i32, i32, P, P, ctypes.POINTER(pa.pa_cache_desc),
+                                     P, i32, P, i32, F, i32, P]
+    lib.pa_decode_static.restype = E
+    fake = P(0x10000)
+    desc = _desc()
+    assert lib.pa_decode_static(fake, 0, fake, 0, 4, 2, fake, fake, None, fake, 8, fake, 100,
+                                0.125, 0, None) == 1
+    # 4096 rows x 32 heads x 20 partitions of partials: far past 32 MiB
+    big = _desc(num_kv_heads=8, head_dim=128, num_blocks=4096)
+    assert lib.pa_decode_static(fake, 0, fake, 0, 4096, 32, fake, fake, ctypes.byref(big), fake,
+                                160, fake, 2560, 0.125, 128, None) == 3
+    opts = pa.pa_attn_options(window=0, alibi_slopes=0x10002)
+    assert lib.pa_varlen_ex(fake, 0, fake, 0, 10, 2, 2, fake, fake, 5, 100, fake, fake,
+                            ctypes.byref(desc), fake, 8, 0.125, ctypes.byref(opts), fake, 1 << 40,
+                            None) == 1
